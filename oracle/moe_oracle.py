@@ -224,46 +224,55 @@ def layer_backward(fwd: dict, dY, X, W_gu, W_d, k: int) -> dict:
 
 
 # ----------------------------------------------------------- sampled (large sizes)
-def token_forward(tokens, idx, w, X, W_gu, W_d) -> np.ndarray:
-    """Y rows for a subset of tokens, one (token, expert) pair at a time, given
-    the routing (idx, w) of the whole batch. Used where the full oracle is too
-    slow: every output row depends only on its own token's pairs."""
-    X = _f64(X)
-    out = np.zeros((len(tokens), X.shape[1]))
+def _pairs_by_expert(tokens, idx):
+    """(row in the sample, slot j) pairs of the sampled tokens, grouped by expert."""
+    groups = {}
     for n, t in enumerate(tokens):
         for j in range(idx.shape[1]):
-            e = int(idx[t, j])
-            Wgu = _f64(W_gu[e])
-            Wd = _f64(W_d[e])
-            _, _, _, o = expert_mlp(X[t:t + 1], Wgu, Wd)
-            out[n] += w[t, j] * o[0]
+            groups.setdefault(int(idx[t, j]), []).append((n, j))
+    return groups
+
+
+def token_forward(tokens, idx, w, X, W_gu, W_d) -> np.ndarray:
+    """Y rows for a subset of tokens given the routing (idx, w) of the whole
+    batch. Every output row depends only on its own token's pairs, so this is
+    exact for the sampled rows; the pairs are visited expert by expert."""
+    tokens = [int(t) for t in tokens]
+    Xs = _f64(X[tokens])
+    out = np.zeros((len(tokens), Xs.shape[1]))
+    for e, pairs in sorted(_pairs_by_expert(tokens, idx).items()):
+        n = np.array([a for a, _ in pairs])
+        j = np.array([b for _, b in pairs])
+        _, _, _, o = expert_mlp(Xs[n], _f64(W_gu[e]), _f64(W_d[e]))
+        wt = np.asarray(w)[np.asarray(tokens)[n], j]
+        np.add.at(out, n, wt[:, None] * o)
     return out
 
 
 def token_backward(tokens, idx, w, probs, dY, X, W_gu, W_d) -> dict:
     """dX and d logits rows for a subset of tokens (each depends only on the
     token's own pairs), with the same formulas as ``layer_backward``."""
-    X = _f64(X)
-    dY = _f64(dY)
-    H = X.shape[1]
-    k = idx.shape[1]
-    dX = np.zeros((len(tokens), H))
-    dw = np.zeros((len(tokens), k))
-    for n, t in enumerate(tokens):
-        for j in range(k):
-            e = int(idx[t, j])
-            Wgu = _f64(W_gu[e])
-            Wd = _f64(W_d[e])
-            I = Wd.shape[1]
-            g, u, h, o = expert_mlp(X[t:t + 1], Wgu, Wd)
-            dw[n, j] = float((dY[t:t + 1] * o).sum())
-            dh = (w[t, j] * dY[t:t + 1]) @ Wd
-            s = sigmoid(g)
-            du = dh * g * s
-            dg = dh * u * s * (1.0 + g * (1.0 - s))
-            dX[n] += (dg @ Wgu[:I] + du @ Wgu[I:])[0]
+    tokens = [int(t) for t in tokens]
     tk = np.asarray(tokens)
-    dlogits = router_backward(dw, w[tk], probs[tk], np.asarray(idx)[tk])
+    Xs = _f64(X[tokens])
+    dYs = _f64(dY[tokens])
+    k = idx.shape[1]
+    dX = np.zeros_like(Xs)
+    dw = np.zeros((len(tokens), k))
+    for e, pairs in sorted(_pairs_by_expert(tokens, idx).items()):
+        n = np.array([a for a, _ in pairs])
+        j = np.array([b for _, b in pairs])
+        Wgu = _f64(W_gu[e])
+        Wd = _f64(W_d[e])
+        I = Wd.shape[1]
+        g, u, h, o = expert_mlp(Xs[n], Wgu, Wd)
+        dw[n, j] = (dYs[n] * o).sum(axis=1)
+        dh = (np.asarray(w)[tk[n], j][:, None] * dYs[n]) @ Wd
+        s = sigmoid(g)
+        du = dh * g * s
+        dg = dh * u * s * (1.0 + g * (1.0 - s))
+        np.add.at(dX, n, dg @ Wgu[:I] + du @ Wgu[I:])
+    dlogits = router_backward(dw, np.asarray(w)[tk], np.asarray(probs)[tk], np.asarray(idx)[tk])
     return dict(dX=dX, dlogits=dlogits, dw=dw)
 
 

@@ -1,0 +1,195 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) fused MoE expert layer.
+ *
+ * The layer replaces the for-loop over experts of Hugging Face MoE blocks
+ * ("Integration of fused moe kernel (e.g., megablocks) for efficient moe
+ * training", axolotl issue #3155, Feature description) with routed grouped
+ * GEMMs:
+ *
+ *   logits [T,E] --moe_route--> top-k ids/weights --moe_permute--> counts,
+ *   offsets, expert-sorted pair order, gathered rows Xp --moe_experts_fwd-->
+ *   SwiGLU(gate/up) and down per expert segment, routing weight applied -->
+ *   moe_combine --> Y [T,H];  moe_layer_bwd gives dX, dW_gate/up/down and
+ *   d router logits.
+ *
+ * Notation: T tokens, H hidden size, E experts, k experts per token, I expert
+ * intermediate size, P = T*k (token, expert) pairs. Pair id q = t*k + j where
+ * j is the rank of the expert in token t's top-k (descending score). Row r of
+ * every permuted buffer holds pair sorted_pair[r]; the rows of expert e are
+ * [offsets[e], offsets[e+1]).
+ *
+ * Conventions shared by every call:
+ *  - Memory: every pointer is a DEVICE pointer owned by the caller, row-major
+ *    and contiguous, 16-byte aligned. The library allocates no device memory
+ *    and keeps no pointer after a call returns; scratch space is the caller's
+ *    `ws` buffer, sized by the matching *_workspace_bytes query.
+ *  - Types: bf16 tensors are passed as moe_bf16 (the raw 16-bit pattern);
+ *    index tensors are int32; weights/logits/gradients of the router are fp32.
+ *  - Streams: each call only enqueues work on `stream` (NULL = legacy default
+ *    stream) and returns without synchronising. Nothing is read back to the
+ *    host; the per-expert counts never leave the device.
+ *  - Errors: arguments are checked before anything is launched. A bad shape,
+ *    a NULL required pointer or a pointer that is not 16-byte aligned returns
+ *    MOE_ERR_INVALID_ARG, a workspace that is too small MOE_ERR_WORKSPACE, a
+ *    device that is not sm_100 MOE_ERR_UNSUPPORTED, a failed launch
+ *    MOE_ERR_CUDA. Problems found on the device (an expert id outside [0,E),
+ *    a pipeline wait that exceeded its time limit) are recorded in a device
+ *    status word that moe_last_device_status reads; kernels never trap.
+ *  - Limits: 1 <= k <= E <= 1024, T >= 0 (T == 0 is a valid empty batch),
+ *    T*k < 2^31, H and I positive multiples of 8 (16-byte rows).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;                 /* bfloat16 bit pattern */
+typedef struct CUstream_st* moe_stream_t;  /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_TIMEOUT = 5,
+  MOE_ERR_DEVICE_CHECK = 6
+} moe_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_str(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: MOE_OK, MOE_ERR_TIMEOUT (a kernel wait ran out and the
+ * kernel unwound) or MOE_ERR_DEVICE_CHECK (an expert id outside [0,E) was
+ * skipped). MOE_ERR_CUDA if the synchronisation itself failed. */
+int moe_last_device_status(moe_stream_t stream);
+
+/*
+ * moe_route -- router softmax, top-k, renormalisation.
+ * Source: fused-MoE Triton project summary (sourcepulse), Highlighted
+ * Details ("fused softmax-topk"); "[WIP] Qwen3 MoE support" (torchtune PR
+ * #2820), review comment: the top-k scores are divided by their sum + 1e-20.
+ *
+ *   p[t,:]       = softmax(logits[t,:])             (fp32)
+ *   topk_idx[t,:] = the k experts with the largest logits, ordered by logit
+ *                   descending, ties to the lower expert index (the set is
+ *                   the top-k of p because softmax is increasing)
+ *   topk_w[t,j]  = p[t,idx_j] / (sum_j' p[t,idx_j'] + 1e-20)
+ *
+ * logits   [T,E] fp32 in.      topk_idx [T,k] int32 out.
+ * topk_w   [T,k] fp32 out.     probs    [T,E] fp32 out, or NULL to skip
+ *                              (moe_layer_bwd needs it).
+ */
+int moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w, float* probs,
+              moe_stream_t stream);
+
+/* Bytes of workspace moe_permute needs for this problem size. */
+size_t moe_permute_workspace_bytes(int T, int E, int k);
+
+/*
+ * moe_permute -- per-expert histogram, prefix sum and stable scatter that
+ * sorts the P pairs by expert, plus the row gather Xp[r] = X[sorted_pair[r]/k].
+ * Source: "[MoE] Improve moe kernels for unsloth fine tuning #3812", review
+ * of the token-routing logic: counts = bincount(flat expert ids, minlength=E)
+ * (one value per expert) and gather indices = stable argsort of the flat ids;
+ * fused-MoE summary, How It Works: inputs sorted by expert.
+ *
+ * topk_idx    [T,k] int32 in (values in [0,E); others are skipped and flagged
+ *             as MOE_ERR_DEVICE_CHECK in the device status word).
+ * counts      [E] int32 out;  offsets [E+1] int32 out (exclusive prefix sum).
+ * sorted_pair [P] int32 out: pair ids in expert order, ascending pair id
+ *             within an expert (bit-identical to a stable argsort).
+ * pair_pos    [P] int32 out: inverse permutation, pair_pos[sorted_pair[r]] = r.
+ * X [T,H] bf16 in and Xp [P,H] bf16 out: the gather; both NULL to skip it
+ *             (H is then ignored).
+ * ws          >= moe_permute_workspace_bytes(T,E,k) bytes of device scratch.
+ */
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X, int H, moe_bf16* Xp, void* ws,
+                size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_experts_fwd -- the two persistent grouped GEMMs over the expert
+ * segments (tcgen05 tensor cores, TMEM accumulators, TMA-fed tiles; experts
+ * with no rows cost nothing).
+ * Source: fused-MoE summary, How It Works (grouped GEMM with persistent
+ * workers over expert-sorted rows); unsloth PR #3812, stacked weight shapes
+ * and the fused post-multiply by the routing weight ("fuse_mul_post").
+ *
+ *   gate/up:  g = Xp[r] W_gu[e,0:I]^T,  u = Xp[r] W_gu[e,I:2I]^T  (fp32 acc)
+ *             h[r] = silu(g) * u  -> bf16          (SwiGLU in the epilogue)
+ *   down:     O[r] = w_q * (h[r] W_d[e]^T)  -> bf16 (weight in the epilogue)
+ *   with q = sorted_pair[r], w_q = topk_w[q] (topk_w NULL: w_q = 1).
+ *
+ * Xp [P,H] bf16 in; offsets [E+1], sorted_pair [P] int32 in (moe_permute).
+ * W_gu [E,2I,H] bf16: rows 0..I-1 gate, I..2I-1 up (Linear [out,in] layout).
+ * W_d  [E,H,I]  bf16.
+ * h [P,I] bf16 out; gu_save [P,2I] bf16 out (g then u per row) or NULL;
+ * O [P,H] bf16 out. Rows of Xp/h/O past P are never touched.
+ */
+int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream);
+
+/*
+ * moe_combine -- un-permute and sum each token's k results:
+ *   Y[t] = sum_{j=0..k-1} O[pair_pos[t*k+j]], summed in fp32 in j order,
+ *   rounded once to bf16.
+ * Source: modelopt moe helpers, a2a_moe Flow (weight by the routing weights
+ * and sum each token's top-k results; results return in the hidden dtype).
+ * O [P,H] bf16 in; pair_pos [P] int32 in; Y [T,H] bf16 out.
+ */
+int moe_combine(const moe_bf16* O, const int32_t* pair_pos, int T, int k, int H, moe_bf16* Y,
+                moe_stream_t stream);
+
+/* Bytes of workspace moe_layer_bwd needs; recompute_gu != 0 adds room to
+ * recompute the gate/up activations when gu_save is not available. */
+size_t moe_layer_bwd_workspace_bytes(int T, int E, int k, int H, int I, int recompute_gu);
+
+/*
+ * moe_layer_bwd -- backward of route -> experts -> combine for upstream
+ * gradient dY, with the top-k selection held constant. The pages give no
+ * backward formulas; these are the derivatives of the forward above:
+ *   dw_q      = <dY[t], h[r] W_d[e]^T>                  (d routing weight)
+ *   dh[r]     = w_q * dY[t] W_d[e]
+ *   du, dg    = dh*silu(g),  dh*u*s*(1+g*(1-s)), s = sigmoid(g)
+ *   dW_d[e]   = sum_r (w_q dY[t])^T h[r];  dW_gu[e] = sum_r [dg;du]^T Xp[r]
+ *   dX[t]     = sum_j [dg;du][pair_pos[t*k+j]] W_gu[e]
+ *   dlogits   = softmax Jacobian of (renormalisation Jacobian of dw)
+ * Experts with no rows get exactly zero dW.
+ *
+ * dY [T,H] bf16 in. Xp, h, offsets, sorted_pair, pair_pos, topk_idx, topk_w
+ * and probs as produced by the forward calls. gu_save [P,2I] from
+ * moe_experts_fwd, or NULL to recompute it (needs recompute_gu workspace).
+ * Outputs: dX [T,H] bf16, dW_gu [E,2I,H] bf16, dW_d [E,H,I] bf16,
+ * dlogits [T,E] fp32. ws >= moe_layer_bwd_workspace_bytes(...).
+ */
+int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Per-kernel timing with CUDA events recorded on the launching stream around
+ * every kernel launch (off by default; measurement only, no effect on results).
+ * moe_profile_enable(1) starts recording and clears earlier records.
+ * moe_profile_read synchronises on the recorded events and returns the total
+ * device milliseconds and launch count of kernel `name` (see
+ * moe_profile_kernel_name); MOE_ERR_INVALID_ARG for an unknown name.
+ */
+int moe_profile_enable(int on);
+int moe_profile_read(const char* name, double* total_ms, int* launches);
+/* Name of kernel slot i (0-based), NULL past the last one. */
+const char* moe_profile_kernel_name(int i);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,213 @@
+"""Thin ctypes binding of the C ABI in include/moe.h.
+
+Each function has the C call's name and only marshals arguments: it checks
+dtypes/shapes/devices of the torch tensors, allocates missing outputs with
+torch (the library itself never allocates) and passes raw pointers and the
+current CUDA stream. Every step of the layer runs in the CUDA library; when
+the library is missing this module raises instead of computing anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+_LIB = None
+_c_void = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_size = ctypes.c_size_t
+
+_SIGNATURES = {
+    "moe_status_str": (ctypes.c_char_p, [_c_int]),
+    "moe_last_device_status": (_c_int, [_c_void]),
+    "moe_route": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void]),
+    "moe_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "moe_permute": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void, _c_void,
+                             _c_int, _c_void, _c_void, _c_size, _c_void]),
+    "moe_experts_fwd": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                 _c_void, _c_void, _c_void, _c_void, _c_void, _c_void]),
+    "moe_combine": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void]),
+    "moe_layer_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 7 + [_c_void, _c_size, _c_void]),
+    "moe_profile_enable": (_c_int, [_c_int]),
+    "moe_profile_read": (_c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
+    "moe_profile_kernel_name": (ctypes.c_char_p, [_c_int]),
+}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {status_str(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libmoe.so (building it first when nvcc is available)."""
+    global _LIB
+    if _LIB is None:
+        path = _build.LIB_PATH
+        if not _build.up_to_date():
+            _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError("libmoe.so is not built; the MoE layer has no other implementation")
+        l = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = l
+    return _LIB
+
+
+def header_symbols() -> list[str]:
+    """Function names declared in include/*.h."""
+    names = []
+    for f in sorted(os.listdir(_build.INCLUDE)):
+        if f.endswith(".h"):
+            text = open(os.path.join(_build.INCLUDE, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def status_str(status: int) -> str:
+    return lib().moe_status_str(status).decode()
+
+
+def _check(call: str, status: int):
+    if status != 0:
+        raise MoeError(call, status)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def last_device_status(stream=None) -> int:
+    return lib().moe_last_device_status(_stream(stream))
+
+
+# ------------------------------------------------------------------- calls
+def moe_route(logits: torch.Tensor, k: int, topk_idx=None, topk_w=None, probs=None, want_probs=True, stream=None):
+    T, E = logits.shape
+    dev = logits.device
+    _need(logits, torch.float32, (T, E), "logits")
+    topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty(T, k, dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    if probs is None and want_probs:
+        probs = torch.empty(T, E, dtype=torch.float32, device=dev)
+    _check("moe_route", lib().moe_route(_ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _ptr(probs),
+                                        _stream(stream)))
+    return topk_idx, topk_w, probs
+
+
+def moe_permute(topk_idx: torch.Tensor, E: int, X: torch.Tensor | None = None, out=None, ws=None, stream=None):
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    P = T * k
+    o = dict(out or {})
+    o.setdefault("counts", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    o.setdefault("sorted_pair", torch.empty(P, dtype=torch.int32, device=dev))
+    o.setdefault("pair_pos", torch.empty(P, dtype=torch.int32, device=dev))
+    H = 0
+    if X is not None:
+        H = X.shape[1]
+        _need(X, torch.bfloat16, (T, H), "X")
+        o.setdefault("Xp", torch.empty(P, H, dtype=torch.bfloat16, device=dev))
+    need = lib().moe_permute_workspace_bytes(T, E, k)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("moe_permute", lib().moe_permute(
+        _ptr(topk_idx), T, E, k, _ptr(o["counts"]), _ptr(o["offsets"]), _ptr(o["sorted_pair"]),
+        _ptr(o["pair_pos"]), _ptr(X), H, _ptr(o.get("Xp")), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_experts_fwd(Xp, offsets, sorted_pair, topk_w, T, E, k, W_gu, W_d, h=None, gu_save=None, O=None,
+                    save_gu=True, stream=None):
+    P = T * k
+    H = W_gu.shape[2]
+    I = W_d.shape[2]
+    dev = Xp.device
+    _need(Xp, torch.bfloat16, (P, H), "Xp")
+    _need(W_gu, torch.bfloat16, (E, 2 * I, H), "W_gu")
+    _need(W_d, torch.bfloat16, (E, H, I), "W_d")
+    h = torch.empty(P, I, dtype=torch.bfloat16, device=dev) if h is None else h
+    if gu_save is None and save_gu:
+        gu_save = torch.empty(P, 2 * I, dtype=torch.bfloat16, device=dev)
+    O = torch.empty(P, H, dtype=torch.bfloat16, device=dev) if O is None else O
+    _check("moe_experts_fwd", lib().moe_experts_fwd(
+        _ptr(Xp), _ptr(offsets), _ptr(sorted_pair), _ptr(topk_w), T, E, k, H, I, _ptr(W_gu), _ptr(W_d),
+        _ptr(h), _ptr(gu_save), _ptr(O), _stream(stream)))
+    return h, gu_save, O
+
+
+def moe_combine(O, pair_pos, T, k, Y=None, stream=None):
+    H = O.shape[1]
+    Y = torch.empty(T, H, dtype=torch.bfloat16, device=O.device) if Y is None else Y
+    _check("moe_combine", lib().moe_combine(_ptr(O), _ptr(pair_pos), T, k, H, _ptr(Y), _stream(stream)))
+    return Y
+
+
+def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
+                  W_gu, W_d, out=None, ws=None, stream=None):
+    H = W_gu.shape[2]
+    I = W_d.shape[2]
+    dev = dY.device
+    o = dict(out or {})
+    o.setdefault("dX", torch.empty(T, H, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW_d", torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dlogits", torch.empty(T, E, dtype=torch.float32, device=dev))
+    need = lib().moe_layer_bwd_workspace_bytes(T, E, k, H, I, 1 if gu_save is None else 0)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("moe_layer_bwd", lib().moe_layer_bwd(
+        _ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
+        _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]),
+        _ptr(o["dW_gu"]), _ptr(o["dW_d"]), _ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+# --------------------------------------------------------------- profiling
+def profile_enable(on: bool = True):
+    _check("moe_profile_enable", lib().moe_profile_enable(1 if on else 0))
+
+
+def profile_kernel_names() -> list[str]:
+    names, i = [], 0
+    while True:
+        n = lib().moe_profile_kernel_name(i)
+        if n is None:
+            return names
+        names.append(n.decode())
+        i += 1
+
+
+def profile_read() -> dict:
+    """{kernel name: (total device ms, launches)} of the recorded launches."""
+    out = {}
+    for n in profile_kernel_names():
+        ms = ctypes.c_double()
+        cnt = ctypes.c_int()
+        _check("moe_profile_read", lib().moe_profile_read(n.encode(), ctypes.byref(ms), ctypes.byref(cnt)))
+        if cnt.value:
+            out[n] = (ms.value, cnt.value)
+    return out

@@ -1,0 +1,519 @@
+// Persistent grouped GEMM over variable-size expert segments for sm_100a.
+//
+// fused-MoE Triton project summary, How It Works: one grouped GEMM with
+// persistent workers over expert-sorted rows replaces the per-expert loop;
+// unsloth PR #3812: stacked expert weights [E, 2I, H] / [E, H, I] and the
+// routing-weight multiply fused after the GEMM ("fuse_mul_post").
+//
+// B200 design (not a translation of the Triton kernels):
+//  * one CTA per SM, 6 warps: warp 0 issues TMA loads, warp 1 issues tcgen05
+//    MMAs (and owns the TMEM allocation), warps 2-5 run the epilogue;
+//  * 128 x 256 output tiles, K staged 64 at a time through a 4-deep ring of
+//    128-byte-swizzled shared-memory tiles fed by TMA, synchronised with
+//    mbarriers (TMA -> MMA "full", MMA commit -> TMA "empty");
+//  * the fp32 accumulator lives in TMEM, double-buffered (2 x 256 columns),
+//    so the epilogue of tile i overlaps the main loop of tile i+1;
+//  * the tile list is built on the device from the per-expert offsets, so the
+//    host never learns the counts and experts without rows cost nothing.
+//
+// Variants (all D = A * B^T with bf16 operands and fp32 accumulation):
+//  FwdGateUp   A = Xp[P,H] (K-major), B = W_gu[e] gate rows and up rows
+//              interleaved per tile (128 + 128), epilogue h = silu(g) * u.
+//  FwdDown     A = h[P,I], B = W_d[e][H,I], epilogue O = w_q * acc.
+//  BwdDgradDown   A = dYp[P,H], B = W_d[e] read MN-major ([H,I] as K x N);
+//              epilogue: partial dw = <acc, h>, dh = w_q*acc, SwiGLU backward
+//              -> dGU = [dg | du], and hw = w_q * h for the down wgrad.
+//  BwdDgradGateUp A = dGU[P,2I], B = W_gu[e] MN-major ([2I,H] as K x N) -> dXp.
+//  BwdWgrad    per expert dW[e] = A^T B with the expert's rows as K; both
+//              operands MN-major; the last K block of a segment is clipped
+//              by zeroing the rows past the segment in shared memory.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+
+enum GemmKind : int { kFwdGateUp = 0, kFwdDown = 1, kBwdDgradDown = 2, kBwdDgradGateUp = 3, kBwdWgrad = 4 };
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kUmmaK = 16;
+constexpr int kStages = 4;
+constexpr int kATileBytes = kBM * kBK * 2;  // 16 KiB
+constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KiB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 2 * kBN;
+constexpr int kMaxExperts = 1024;
+constexpr int kNumBarriers = 2 * kStages + 5;
+
+struct GemmParams {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  const int32_t* offsets;      // [E+1] expert segment bounds in the permuted rows
+  const int32_t* sorted_pair;  // [P]
+  const float* topk_w;         // [P] routing weight per pair id (NULL: 1)
+  int64_t P;
+  int E;
+  int N;        // output columns: I (gate/up), H (down), I (dgrad-down), H (dgrad-gate/up), N (wgrad)
+  int K;        // reduction length of the row-grouped variants
+  int M;        // wgrad: rows of dW[e]
+  int I;        // intermediate size (gate/up row split)
+  int b_rows;   // rows of the B tensor map that belong to one expert
+  int n_tiles;  // tiles along N
+  int m_tiles;  // wgrad: tiles along M
+  uint16_t* out;             // output (bf16), row stride out_ld
+  int64_t out_ld;
+  int64_t out_expert_stride;  // wgrad: elements per expert
+  uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
+  const uint16_t* h_in;       // BwdDgradDown: h
+  uint16_t* hw_out;           // BwdDgradDown: w_q * h
+  float* dw_part;             // BwdDgradDown: [P, n_tiles] partial routing-weight grads
+};
+
+__host__ __device__ inline size_t gemm_smem_bytes(int E) {
+  return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes + kNumBarriers * 8 + 16 +
+         2 * static_cast<size_t>(E + 1) * 4;
+}
+
+struct TileInfo {
+  int e, m_blk, n_blk;
+  int row0;     // first permuted row (row-grouped) / first K row (wgrad)
+  int rows;     // valid rows in the tile (row-grouped) / rows of the segment (wgrad)
+  int num_kb;   // K blocks
+};
+
+template <int KIND>
+__device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
+                                                const int* s_tstart) {
+  TileInfo ti;
+  if constexpr (KIND == kBwdWgrad) {
+    const int per_e = p.m_tiles * p.n_tiles;
+    ti.e = t / per_e;
+    const int local = t - ti.e * per_e;
+    ti.m_blk = local / p.n_tiles;
+    ti.n_blk = local - ti.m_blk * p.n_tiles;
+    ti.row0 = s_off[ti.e];
+    ti.rows = s_off[ti.e + 1] - ti.row0;
+    ti.num_kb = (ti.rows + kBK - 1) / kBK;
+  } else {
+    int lo = 0, hi = p.E;  // s_tstart[lo] <= t < s_tstart[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tstart[mid] <= t) lo = mid; else hi = mid;
+    }
+    ti.e = lo;
+    const int local = t - s_tstart[lo];
+    ti.m_blk = local / p.n_tiles;
+    ti.n_blk = local - ti.m_blk * p.n_tiles;
+    ti.row0 = s_off[lo] + ti.m_blk * kBM;
+    ti.rows = min(kBM, s_off[lo + 1] - ti.row0);
+    ti.num_kb = (p.K + kBK - 1) / kBK;
+  }
+  return ti;
+}
+
+// Bounded wait done by every lane of a warp; the result is warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void store8_bf16(uint16_t* dst, const float* v) {
+  uint4 o;
+  o.x = pack_bf16(v[0], v[1]);
+  o.y = pack_bf16(v[2], v[3]);
+  o.z = pack_bf16(v[4], v[5]);
+  o.w = pack_bf16(v[6], v[7]);
+  *reinterpret_cast<uint4*>(dst) = o;
+}
+
+__device__ __forceinline__ void load8_bf16(const uint16_t* src, float* v) {
+  const uint4 i = *reinterpret_cast<const uint4*>(src);
+  v[0] = bf16lo(i.x); v[1] = bf16hi(i.x);
+  v[2] = bf16lo(i.y); v[3] = bf16hi(i.y);
+  v[4] = bf16lo(i.z); v[5] = bf16hi(i.z);
+  v[6] = bf16lo(i.w); v[7] = bf16hi(i.w);
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+template <int KIND>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr bool kWgrad = (KIND == kBwdWgrad);
+  constexpr bool kAMN = kWgrad;
+  constexpr bool kBMN = (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || kWgrad);
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, kAMN, kBMN);
+  constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
+  constexpr uint32_t kBLbo = kBMN ? 8192u : 16u;
+  constexpr uint32_t kAStep = kAMN ? 2048u : 32u;  // bytes per UMMA_K step
+  constexpr uint32_t kBStep = kBMN ? 2048u : 32u;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kATileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + kStages;
+  uint64_t* tfull_bar = bars + 2 * kStages;
+  uint64_t* tempty_bar = bars + 2 * kStages + 2;
+  uint64_t* drain_bar = bars + 2 * kStages + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBarriers);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_tstart = s_off + (p.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+    }
+    mbar_init(drain_bar, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
+  __syncthreads();
+  if (warp == 0 && !kWgrad) {
+    // tiles of expert e = ceil(rows_e / BM) * n_tiles; exclusive prefix over experts
+    const int per = (p.E + 31) / 32;
+    const int e0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < p.E) local += ((s_off[e + 1] - s_off[e] + kBM - 1) / kBM) * p.n_tiles;
+    }
+    const int incl = warp_inclusive_scan(local);
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < p.E) {
+        s_tstart[e] = run;
+        run += ((s_off[e + 1] - s_off[e] + kBM - 1) / kBM) * p.n_tiles;
+      }
+    }
+    if (lane == 31) s_tstart[p.E] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = kWgrad ? p.E * p.m_tiles * p.n_tiles : s_tstart[p.E];
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
+        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+            report(MOE_ERR_TIMEOUT);
+            *s_abort = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+          uint8_t* a_dst = sA + stage * kATileBytes;
+          uint8_t* b_dst = sB + stage * kBTileBytes;
+          const int kx = kb * kBK;
+          if constexpr (KIND == kFwdGateUp) {
+            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
+            const int gate_row = ti.e * p.b_rows + ti.n_blk * 128;
+            tma_load_2d(b_dst, &p.tmB, &full_bar[stage], kx, gate_row);
+            tma_load_2d(b_dst + 16384, &p.tmB, &full_bar[stage], kx, gate_row + p.I);
+          } else if constexpr (KIND == kFwdDown) {
+            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
+            const int brow = ti.e * p.b_rows + ti.n_blk * kBN;
+            tma_load_2d(b_dst, &p.tmB, &full_bar[stage], kx, brow);
+            tma_load_2d(b_dst + 16384, &p.tmB, &full_bar[stage], kx, brow + 128);
+          } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
+            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
+            const int krow = ti.e * p.b_rows + kx;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(b_dst + c * 8192, &p.tmB, &full_bar[stage], ti.n_blk * kBN + 64 * c, krow);
+          } else {  // wgrad: K rows are the expert's permuted rows
+            const int krow = ti.row0 + kx;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_load_2d(a_dst + c * 8192, &p.tmA, &full_bar[stage], ti.m_blk * kBM + 64 * c, krow);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(b_dst + c * 8192, &p.tmB, &full_bar[stage], ti.n_blk * kBN + 64 * c, krow);
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Let every load still in flight land before the block may exit
+      // (immediate in normal operation: the consumer has waited on them).
+      const int inflight = issued < kStages ? issued : kStages;
+      for (int i = 0; i < inflight; ++i) {
+        if (--stage < 0) {
+          stage = kStages - 1;
+          phase ^= 1u;
+        }
+        mbar_wait(&full_bar[stage], phase);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int tcount = 0;
+    for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
+      const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+      if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogue writes zeros
+      const int acc = tcount & 1;
+      if (!warp_wait(&tempty_bar[acc], ((tcount >> 1) & 1) ^ 1u)) {
+        if (lane == 0) report(MOE_ERR_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+      bool ok = true;
+      for (int kb = 0; kb < ti.num_kb; ++kb) {
+        if (!warp_wait(&full_bar[stage], phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if constexpr (kWgrad) {
+          const int valid = ti.rows - kb * kBK;
+          if (valid < kBK) {
+            // rows past the segment belong to the next expert: zero them in
+            // both 64-column chunks of the A tile (whole 128-byte rows, so the
+            // swizzle does not matter)
+            uint8_t* a_tile = sA + stage * kATileBytes;
+            const int nrows = kBK - valid;
+            for (int i = lane; i < 2 * nrows * 8; i += 32) {
+              const int chunk = i / (nrows * 8);
+              const int rem = i - chunk * nrows * 8;
+              const int r = valid + rem / 8;
+              const int v16 = rem & 7;
+              *reinterpret_cast<uint4*>(a_tile + chunk * 8192 + r * 128 + v16 * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(sA + stage * kATileBytes);
+          const uint32_t b_addr = smem_u32(sB + stage * kBTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+            const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
+            const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);
+        }
+        __syncwarp();
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        if (lane == 0) report(MOE_ERR_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+      if (lane == 0) umma_commit(&tfull_bar[acc]);
+      __syncwarp();
+      ++tcount;
+    }
+    // all MMAs issued by this warp must finish before TMEM is released
+    if (lane == 0) umma_commit(drain_bar);
+    __syncwarp();
+    warp_wait(drain_bar, 0);
+  } else {
+    // ------------------------------------------------------- epilogue
+    const int sub = warp & 3;           // TMEM sub-partition this warp may access
+    const int row = sub * 32 + lane;    // accumulator row (TMEM lane)
+    int tcount = 0;
+    for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
+      const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+      if constexpr (kWgrad) {
+        if (ti.num_kb == 0) {
+          const int m = ti.m_blk * kBM + row;
+          if (m < p.M) {
+            uint16_t* dst = p.out + ti.e * p.out_expert_stride + static_cast<int64_t>(m) * p.out_ld;
+            for (int c = ti.n_blk * kBN; c < min(p.N, ti.n_blk * kBN + kBN); c += 8)
+              *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);
+          }
+          continue;
+        }
+      }
+      const int acc = tcount & 1;
+      if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
+        if (lane == 0) report(MOE_ERR_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(sub * 32) << 16);
+
+      if constexpr (KIND == kFwdGateUp) {
+        const bool rvalid = row < ti.rows;
+        const int64_t r = ti.row0 + row;
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(taddr + c, g);
+          tmem_ld_32x32b_x32(taddr + 128 + c, u);
+          tmem_ld_wait();
+          const int i0 = ti.n_blk * 128 + c;
+          if (rvalid && i0 < p.I) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (i0 + 8 * v < p.I) {
+                float hv[8], gv[8], uv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  gv[j] = __uint_as_float(g[8 * v + j]);
+                  uv[j] = __uint_as_float(u[8 * v + j]);
+                  hv[j] = silu_f(gv[j]) * uv[j];
+                }
+                if (p.out != nullptr) store8_bf16(p.out + r * p.out_ld + i0 + 8 * v, hv);
+                if (p.gu != nullptr) {
+                  store8_bf16(p.gu + r * (2 * p.I) + i0 + 8 * v, gv);
+                  store8_bf16(p.gu + r * (2 * p.I) + p.I + i0 + 8 * v, uv);
+                }
+              }
+            }
+          }
+        }
+      } else if constexpr (KIND == kFwdDown || KIND == kBwdDgradGateUp) {
+        const bool rvalid = row < ti.rows;
+        const int64_t r = ti.row0 + row;
+        float wq = 1.0f;
+        if constexpr (KIND == kFwdDown) {
+          if (rvalid && p.topk_w != nullptr) {
+            const int32_t q = p.sorted_pair[r];
+            wq = (q >= 0 && q < p.P) ? p.topk_w[q] : 0.0f;
+          }
+        }
+        for (int c = 0; c < kBN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(taddr + c, a);
+          tmem_ld_wait();
+          const int n0 = ti.n_blk * kBN + c;
+          if (rvalid && n0 < p.N) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + 8 * v < p.N) {
+                float o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = wq * __uint_as_float(a[8 * v + j]);
+                store8_bf16(p.out + r * p.out_ld + n0 + 8 * v, o);
+              }
+            }
+          }
+        }
+      } else if constexpr (KIND == kBwdDgradDown) {
+        const bool rvalid = row < ti.rows;
+        const int64_t r = ti.row0 + row;
+        float wq = 0.0f;
+        if (rvalid) {
+          const int32_t q = p.sorted_pair[r];
+          wq = (q >= 0 && q < p.P) ? p.topk_w[q] : 0.0f;
+        }
+        float dwp = 0.0f;
+        const int I = p.I;
+        for (int c = 0; c < kBN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(taddr + c, a);
+          tmem_ld_wait();
+          const int i0 = ti.n_blk * kBN + c;
+          if (rvalid && i0 < I) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int i = i0 + 8 * v;
+              if (i < I) {
+                float gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
+                load8_bf16(p.gu + r * (2 * I) + i, gv);
+                load8_bf16(p.gu + r * (2 * I) + I + i, uv);
+                load8_bf16(p.h_in + r * I + i, hv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float dhp = __uint_as_float(a[8 * v + j]);
+                  dwp += dhp * hv[j];
+                  const float dh = wq * dhp;
+                  const float s = sigmoid_f(gv[j]);
+                  du[j] = dh * gv[j] * s;
+                  dg[j] = dh * uv[j] * s * (1.0f + gv[j] * (1.0f - s));
+                  hw[j] = wq * hv[j];
+                }
+                store8_bf16(p.out + r * p.out_ld + i, dg);
+                store8_bf16(p.out + r * p.out_ld + I + i, du);
+                store8_bf16(p.hw_out + r * I + i, hw);
+              }
+            }
+          }
+        }
+        if (rvalid) p.dw_part[r * p.n_tiles + ti.n_blk] = dwp;
+      } else {  // wgrad
+        const int m = ti.m_blk * kBM + row;
+        const bool mvalid = m < p.M;
+        uint16_t* dst = p.out + ti.e * p.out_expert_stride + static_cast<int64_t>(m) * p.out_ld;
+        for (int c = 0; c < kBN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(taddr + c, a);
+          tmem_ld_wait();
+          const int n0 = ti.n_blk * kBN + c;
+          if (mvalid && n0 < p.N) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + 8 * v < p.N) {
+                float o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(a[8 * v + j]);
+                store8_bf16(dst + n0 + 8 * v, o);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      ++tcount;
+    }
+  }
+
+  // ------------------------------------------------------------- tear-down
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

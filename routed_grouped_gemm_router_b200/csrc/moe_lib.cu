@@ -1,0 +1,554 @@
+// C ABI of the fused MoE expert layer (declared in include/moe.h).
+//
+// This file validates arguments, sizes the caller's workspace, encodes the TMA
+// tensor maps and enqueues the kernels of route.cuh, permute.cuh,
+// grouped_gemm.cuh, combine.cuh and router_bwd.cuh on the caller's stream.
+// It allocates no device memory and never synchronises (except the status
+// read and the profiling read, which say so).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "combine.cuh"
+#include "common.cuh"
+#include "grouped_gemm.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+#include "router_bwd.cuh"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------------------------ helpers
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+inline bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+constexpr int kMaxDevices = 64;
+
+// Device facts, looked up once per device.
+struct DeviceInfo {
+  int checked = 0;
+  int supported = 0;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.checked = 1;
+  }
+  *out = &d;
+  return d.supported ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// bf16 2-D row-major tensor [rows, inner], 128-byte swizzled boxes of
+// box_inner x box_rows; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+              uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- profiling
+enum ProfSlot : int {
+  kProfRoute = 0,
+  kProfPermCount,
+  kProfPermScan,
+  kProfPermScatter,
+  kProfGatherX,
+  kProfFwdGateUp,
+  kProfFwdDown,
+  kProfCombineY,
+  kProfGatherDy,
+  kProfRecomputeGateUp,
+  kProfDgradDown,
+  kProfDgradGateUp,
+  kProfCombineDx,
+  kProfWgradGateUp,
+  kProfWgradDown,
+  kProfRouterBwd,
+  kProfSlots
+};
+const char* const kProfNames[kProfSlots] = {
+    "route",          "permute_count",       "permute_scan",           "permute_scatter",
+    "gather_x",       "gemm_fwd_gate_up",    "gemm_fwd_down",          "combine_y",
+    "gather_dy",      "gemm_recompute_gate_up", "gemm_bwd_dgrad_down", "gemm_bwd_dgrad_gate_up",
+    "combine_dx",     "gemm_bwd_wgrad_gate_up", "gemm_bwd_wgrad_down", "router_bwd"};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> recs[kProfSlots];
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t take() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void clear() {
+    for (auto& v : recs) {
+      for (auto& pr : v) {
+        pool.push_back(pr.first);
+        pool.push_back(pr.second);
+      }
+      v.clear();
+    }
+  }
+};
+Profiler g_prof;
+
+// Brackets one kernel launch with events on its stream when profiling is on.
+struct ProfScope {
+  int slot;
+  cudaStream_t s;
+  cudaEvent_t end = nullptr;
+  ProfScope(int slot_, cudaStream_t s_) : slot(slot_), s(s_) {
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    if (!g_prof.on) return;
+    cudaEvent_t start = g_prof.take();
+    end = g_prof.take();
+    cudaEventRecord(start, s);
+    g_prof.recs[slot].push_back({start, end});
+  }
+  ~ProfScope() {
+    if (end != nullptr) cudaEventRecord(end, s);
+  }
+};
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <int KIND>
+int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
+  const size_t smem = gemm_smem_bytes(p.E);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ProfScope ps(slot, s);
+  grouped_gemm_kernel<KIND><<<grid, kGemmThreads, smem, s>>>(p);
+  return launch_status();
+}
+
+inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// Persistent grid for the row-grouped GEMMs: at most one CTA per SM and no
+// more than the largest possible tile count.
+inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
+  const int64_t bound = (static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles;
+  return static_cast<int>(bound < num_sms ? bound : num_sms);
+}
+
+GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.E = E;
+  p.P = P;
+  p.offsets = offsets;
+  return p;
+}
+
+bool shape_ok(int T, int E, int k) {
+  return T >= 0 && k >= 1 && E >= k && E <= kMaxExperts && static_cast<int64_t>(T) * k < (int64_t(1) << 31);
+}
+bool dims_ok(int H) { return H > 0 && H % 8 == 0; }
+
+struct BwdLayout {
+  size_t dYp, dGU, hw, dXp, dw_part, gu, total;
+};
+BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
+  (void)E;
+  const size_t P = static_cast<size_t>(T) * k;
+  BwdLayout L;
+  size_t off = 0;
+  L.dYp = off; off += round256(P * H * 2);
+  L.dGU = off; off += round256(P * 2 * I * 2);
+  L.hw = off; off += round256(P * I * 2);
+  L.dXp = off; off += round256(P * H * 2);
+  L.dw_part = off; off += round256(P * cdiv(I, kBN) * 4);
+  L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_str(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+int moe_last_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return v;
+}
+
+int moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w, float* probs,
+              moe_stream_t stream) {
+  if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ok_ptr(logits) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_opt(probs)) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  ProfScope ps(kProfRoute, stream);
+  if (launch_route(logits, T, E, k, topk_idx, topk_w, probs, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+size_t moe_permute_workspace_bytes(int T, int E, int k) {
+  if (!shape_ok(T, E, k)) return 0;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  return round256(static_cast<size_t>(perm_num_chunks(P)) * E * 4);
+}
+
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X, int H, moe_bf16* Xp, void* ws,
+                size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  if (!ok_ptr(counts) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
+  const bool gather = (X != nullptr || Xp != nullptr);
+  if (gather && (!dims_ok(H) || (T > 0 && (!ok_ptr(X) || !ok_ptr(Xp))))) return MOE_ERR_INVALID_ARG;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (P > 0 && (!ok_ptr(topk_idx) || !ok_ptr(sorted_pair) || !ok_ptr(pair_pos))) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_permute_workspace_bytes(T, E, k);
+  if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  if (P == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const int nchunks = perm_num_chunks(P);
+  int* chunk_hist = static_cast<int*>(ws);
+  const size_t hist_smem = sizeof(int) * kPermWarps * E;
+  {
+    ProfScope ps(kProfPermCount, stream);
+    permute_count_kernel<<<nchunks, kPermThreads, hist_smem, stream>>>(topk_idx, P, E, chunk_hist);
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  {
+    ProfScope ps(kProfPermScan, stream);
+    permute_scan_kernel<<<1, 1024, 0, stream>>>(chunk_hist, nchunks, E, counts, offsets);
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  {
+    ProfScope ps(kProfPermScatter, stream);
+    permute_scatter_kernel<<<nchunks, kPermThreads, hist_smem, stream>>>(topk_idx, P, E, chunk_hist, offsets,
+                                                                         sorted_pair, pair_pos);
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  if (gather) {
+    ProfScope ps(kProfGatherX, stream);
+    const int64_t want = (P + 7) / 8;
+    const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
+    gather_rows_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X), sorted_pair, P, k, H / 8,
+                                                   reinterpret_cast<uint4*>(Xp));
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
+  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (P == 0) return MOE_OK;
+  if (!ok_ptr(Xp) || !ok_ptr(offsets) || !ok_ptr(sorted_pair) || !ok_opt(topk_w) || !ok_ptr(W_gu) ||
+      !ok_ptr(W_d) || !ok_ptr(h) || !ok_opt(gu_save) || !ok_ptr(O))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+
+  GemmParams gu = base_params(E, P, offsets);
+  if (!make_map(&gu.tmA, Xp, H, P, 64, 128) || !make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
+    return MOE_ERR_CUDA;
+  gu.sorted_pair = sorted_pair;
+  gu.N = I;
+  gu.K = H;
+  gu.I = I;
+  gu.b_rows = 2 * I;
+  gu.n_tiles = cdiv(I, 128);
+  gu.out = h;
+  gu.out_ld = I;
+  gu.gu = gu_save;
+  if (int st = launch_gemm<kFwdGateUp>(gu, rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms), stream, kProfFwdGateUp))
+    return st;
+
+  GemmParams dn = base_params(E, P, offsets);
+  if (!make_map(&dn.tmA, h, I, P, 64, 128) || !make_map(&dn.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 128))
+    return MOE_ERR_CUDA;
+  dn.sorted_pair = sorted_pair;
+  dn.topk_w = topk_w;
+  dn.N = H;
+  dn.K = I;
+  dn.I = I;
+  dn.b_rows = H;
+  dn.n_tiles = cdiv(H, kBN);
+  dn.out = O;
+  dn.out_ld = H;
+  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown);
+}
+
+int moe_combine(const moe_bf16* O, const int32_t* pair_pos, int T, int k, int H, moe_bf16* Y, moe_stream_t stream) {
+  if (T < 0 || k < 1 || static_cast<int64_t>(T) * k >= (int64_t(1) << 31) || !dims_ok(H)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ok_ptr(O) || !ok_ptr(pair_pos) || !ok_ptr(Y)) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  ProfScope ps(kProfCombineY, stream);
+  return launch_combine(O, pair_pos, T, k, H, Y, stream, dev->num_sms) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_layer_bwd_workspace_bytes(int T, int E, int k, int H, int I, int recompute_gu) {
+  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return 0;
+  return bwd_layout(T, E, k, H, I, recompute_gu != 0).total;
+}
+
+int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
+  if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_ptr(h) || !ok_ptr(probs) ||
+                !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(sorted_pair) || !ok_ptr(pair_pos) ||
+                !ok_ptr(W_gu) || !ok_ptr(W_d) || !ok_ptr(dX) || !ok_ptr(dlogits)))
+    return MOE_ERR_INVALID_ARG;
+  const bool recompute = (gu_save == nullptr);
+  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute);
+  if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  const size_t dw_gu_bytes = static_cast<size_t>(E) * 2 * I * H * 2;
+  const size_t dw_d_bytes = static_cast<size_t>(E) * H * I * 2;
+  if (P == 0) {  // no rows: every expert is empty, all weight gradients are zero
+    if (cudaMemsetAsync(dW_gu, 0, dw_gu_bytes, stream) != cudaSuccess ||
+        cudaMemsetAsync(dW_d, 0, dw_d_bytes, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  moe_bf16* dYp = reinterpret_cast<moe_bf16*>(w8 + L.dYp);
+  moe_bf16* dGU = reinterpret_cast<moe_bf16*>(w8 + L.dGU);
+  moe_bf16* hw = reinterpret_cast<moe_bf16*>(w8 + L.hw);
+  moe_bf16* dXp = reinterpret_cast<moe_bf16*>(w8 + L.dXp);
+  float* dw_part = reinterpret_cast<float*>(w8 + L.dw_part);
+  const int nt_dgrad_down = cdiv(I, kBN);
+
+  // 1. dYp[r] = dY[token of row r]
+  {
+    ProfScope ps(kProfGatherDy, stream);
+    const int64_t want = (P + 7) / 8;
+    const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
+    gather_rows_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(dY), sorted_pair, P, k, H / 8,
+                                                   reinterpret_cast<uint4*>(dYp));
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  // 2. g|u when the forward did not keep them
+  const moe_bf16* gu = gu_save;
+  if (recompute) {
+    moe_bf16* gu_ws = reinterpret_cast<moe_bf16*>(w8 + L.gu);
+    GemmParams rc = base_params(E, P, offsets);
+    if (!make_map(&rc.tmA, Xp, H, P, 64, 128) ||
+        !make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
+      return MOE_ERR_CUDA;
+    rc.sorted_pair = sorted_pair;
+    rc.N = I;
+    rc.K = H;
+    rc.I = I;
+    rc.b_rows = 2 * I;
+    rc.n_tiles = cdiv(I, 128);
+    rc.out = nullptr;
+    rc.gu = gu_ws;
+    if (int st = launch_gemm<kFwdGateUp>(rc, rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms), stream,
+                                         kProfRecomputeGateUp))
+      return st;
+    gu = gu_ws;
+  }
+  // 3. dgrad through down + SwiGLU backward: dGU, hw, partial dw
+  {
+    GemmParams bd = base_params(E, P, offsets);
+    if (!make_map(&bd.tmA, dYp, H, P, 64, 128) ||
+        !make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64))
+      return MOE_ERR_CUDA;
+    bd.sorted_pair = sorted_pair;
+    bd.topk_w = topk_w;
+    bd.N = I;
+    bd.K = H;
+    bd.I = I;
+    bd.b_rows = H;
+    bd.n_tiles = nt_dgrad_down;
+    bd.out = dGU;
+    bd.out_ld = 2 * I;
+    bd.gu = const_cast<moe_bf16*>(gu);
+    bd.h_in = h;
+    bd.hw_out = hw;
+    bd.dw_part = dw_part;
+    if (int st = launch_gemm<kBwdDgradDown>(bd, rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms), stream,
+                                            kProfDgradDown))
+      return st;
+  }
+  // 4. dgrad through gate/up: dXp = dGU W_gu[e]
+  {
+    GemmParams bx = base_params(E, P, offsets);
+    if (!make_map(&bx.tmA, dGU, 2 * I, P, 64, 128) ||
+        !make_map(&bx.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 64))
+      return MOE_ERR_CUDA;
+    bx.N = H;
+    bx.K = 2 * I;
+    bx.I = I;
+    bx.b_rows = 2 * I;
+    bx.n_tiles = cdiv(H, kBN);
+    bx.out = dXp;
+    bx.out_ld = H;
+    if (int st = launch_gemm<kBwdDgradGateUp>(bx, rowgrouped_grid(P, E, bx.n_tiles, dev->num_sms), stream,
+                                              kProfDgradGateUp))
+      return st;
+  }
+  // 5. dX[t] = sum_j dXp[pair_pos[t*k+j]]
+  {
+    ProfScope ps(kProfCombineDx, stream);
+    if (launch_combine(dXp, pair_pos, T, k, H, dX, stream, dev->num_sms) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // 6. weight gradients, K = the expert's rows
+  {
+    GemmParams wg = base_params(E, P, offsets);
+    if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64) || !make_map(&wg.tmB, Xp, H, P, 64, 64)) return MOE_ERR_CUDA;
+    wg.M = 2 * I;
+    wg.N = H;
+    wg.I = I;
+    wg.m_tiles = cdiv(2 * I, kBM);
+    wg.n_tiles = cdiv(H, kBN);
+    wg.out = dW_gu;
+    wg.out_ld = H;
+    wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
+    const int tiles = E * wg.m_tiles * wg.n_tiles;
+    if (int st = launch_gemm<kBwdWgrad>(wg, tiles < dev->num_sms ? tiles : dev->num_sms, stream, kProfWgradGateUp))
+      return st;
+  }
+  {
+    GemmParams wd = base_params(E, P, offsets);
+    if (!make_map(&wd.tmA, dYp, H, P, 64, 64) || !make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
+    wd.M = H;
+    wd.N = I;
+    wd.I = I;
+    wd.m_tiles = cdiv(H, kBM);
+    wd.n_tiles = cdiv(I, kBN);
+    wd.out = dW_d;
+    wd.out_ld = I;
+    wd.out_expert_stride = static_cast<int64_t>(H) * I;
+    const int tiles = E * wd.m_tiles * wd.n_tiles;
+    if (int st = launch_gemm<kBwdWgrad>(wd, tiles < dev->num_sms ? tiles : dev->num_sms, stream, kProfWgradDown))
+      return st;
+  }
+  // 7. router logits gradient
+  {
+    ProfScope ps(kProfRouterBwd, stream);
+    int blocks = (T + 7) / 8;
+    if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
+    router_bwd_kernel<<<blocks, 256, sizeof(float) * 8 * E, stream>>>(probs, topk_idx, topk_w, dw_part, pair_pos,
+                                                                       nt_dgrad_down, T, E, k, dlogits);
+    if (launch_status()) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  g_prof.clear();
+  g_prof.on = (on != 0);
+  return MOE_OK;
+}
+
+int moe_profile_read(const char* name, double* total_ms, int* launches) {
+  if (name == nullptr || total_ms == nullptr || launches == nullptr) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  for (int i = 0; i < kProfSlots; ++i) {
+    if (std::strcmp(name, kProfNames[i]) != 0) continue;
+    double sum = 0.0;
+    for (auto& pr : g_prof.recs[i]) {
+      if (cudaEventSynchronize(pr.second) != cudaSuccess) return MOE_ERR_CUDA;
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess) return MOE_ERR_CUDA;
+      sum += ms;
+    }
+    *total_ms = sum;
+    *launches = static_cast<int>(g_prof.recs[i].size());
+    return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+const char* moe_profile_kernel_name(int i) { return (i >= 0 && i < kProfSlots) ? kProfNames[i] : nullptr; }
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// K-RT: router softmax -> top-k -> renormalise, one warp per token.
+//
+// fused-MoE Triton project summary, Highlighted Details: softmax and top-k are
+// fused into one kernel; "[WIP] Qwen3 MoE support" (torchtune PR #2820),
+// review comment: top-k scores are divided by their sum + 1e-20.
+//
+// Lane l holds experts e = l + 32*v (v < VPL) in registers, so the logits row
+// is read once, coalesced. Selection compares the fp32 logits themselves
+// (logit descending, lower expert index on ties), which makes the chosen set
+// and its order exactly reproducible on any processor given the same logits.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                                    float* __restrict__ probs) {
+  const int lane = threadIdx.x & 31;
+  const int warps_per_block = blockDim.x >> 5;
+  for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
+    const float* row = logits + static_cast<int64_t>(t) * E;
+    float l[VPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int e = lane + 32 * v;
+      l[v] = (e < E) ? __ldg(row + e) : -INFINITY;
+      m = fmaxf(m, l[v]);
+    }
+    m = warp_max_f(m);
+    float z[VPL];
+    float zsum = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int e = lane + 32 * v;
+      z[v] = (e < E) ? expf(l[v] - m) : 0.f;
+      zsum += z[v];
+    }
+    zsum = warp_sum_f(zsum);
+    const float inv = 1.0f / zsum;
+    if (probs != nullptr) {
+      float* prow = probs + static_cast<int64_t>(t) * E;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        if (e < E) prow[e] = z[v] * inv;
+      }
+    }
+    // k rounds of a warp-wide argmax over the not-yet-taken experts.
+    uint32_t taken = 0;
+    float psel[VPL];
+    int isel[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      psel[v] = 0.f;
+      isel[v] = 0;
+    }
+    float psum = 0.f;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        const bool avail = (e < E) && !((taken >> v) & 1u);
+        // within a lane e grows with v, so strict > keeps the lower index on ties
+        if (avail && (l[v] > bv || be == 0x7fffffff)) {
+          bv = l[v];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      // owner lane marks the winner taken; every lane learns its probability
+      float pwin = 0.f;
+      if ((be & 31) == lane) {
+        const int vw = be >> 5;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+          if (v == vw) {
+            taken |= 1u << v;
+            pwin = z[v] * inv;
+          }
+      }
+      pwin = __shfl_sync(0xffffffffu, pwin, be & 31);
+      psum += pwin;
+      if ((j & 31) == lane) {
+        const int vj = j >> 5;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+          if (v == vj) {
+            psel[v] = pwin;
+            isel[v] = be;
+          }
+      }
+    }
+    const float denom = psum + 1e-20f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int j = lane + 32 * v;
+      if (j < k) {
+        topk_idx[static_cast<int64_t>(t) * k + j] = isel[v];
+        topk_w[static_cast<int64_t>(t) * k + j] = psel[v] / denom;
+      }
+    }
+  }
+}
+
+// One-pass launch: picks the register width from E.
+inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* idx, float* w, float* probs,
+                                cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int threads = 256;
+  const int warps = threads / 32;
+  int blocks = (T + warps - 1) / warps;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  const int vpl = (E + 31) / 32;
+#define MOE_ROUTE_CASE(V)                                                                    \
+  if (vpl <= V) {                                                                            \
+    route_kernel<V><<<blocks, threads, 0, s>>>(logits, T, E, k, idx, w, probs);             \
+    return cudaGetLastError();                                                               \
+  }
+  MOE_ROUTE_CASE(1)
+  MOE_ROUTE_CASE(2)
+  MOE_ROUTE_CASE(4)
+  MOE_ROUTE_CASE(8)
+  MOE_ROUTE_CASE(16)
+  MOE_ROUTE_CASE(32)
+#undef MOE_ROUTE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

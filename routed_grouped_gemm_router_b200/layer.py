@@ -1,0 +1,82 @@
+"""The whole expert layer as a sequence of the five C-ABI calls.
+
+``forward`` runs moe_route -> moe_permute -> moe_experts_fwd -> moe_combine
+and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. All
+buffers are torch CUDA tensors; nothing here does arithmetic.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import binding as B
+
+
+@dataclass
+class LayerState:
+    T: int
+    E: int
+    k: int
+    topk_idx: torch.Tensor
+    topk_w: torch.Tensor
+    probs: torch.Tensor
+    perm: dict
+    h: torch.Tensor
+    gu: torch.Tensor | None
+    O: torch.Tensor
+    Y: torch.Tensor
+
+
+def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
+            save_gu: bool = True, bufs: dict | None = None, stream=None) -> LayerState:
+    """Y = combine(experts(permute(X, route(logits)))). ``bufs`` may hold
+    preallocated outputs/workspaces (keys as in the returned state)."""
+    b = bufs or {}
+    T, E = logits.shape
+    idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
+    perm = B.moe_permute(idx, E, X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
+    h, gu, O = B.moe_experts_fwd(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k, W_gu, W_d,
+                                 h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"), save_gu=save_gu,
+                                 stream=stream)
+    Y = B.moe_combine(O, perm["pair_pos"], T, k, Y=b.get("Y"), stream=stream)
+    return LayerState(T, E, k, idx, w, probs, perm, h, gu, O, Y)
+
+
+def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, bufs: dict | None = None,
+             stream=None) -> dict:
+    """dX, dW_gu, dW_d, dlogits for upstream gradient dY."""
+    b = bufs or {}
+    p = st.perm
+    return B.moe_layer_bwd(dY, p["Xp"], st.gu, st.h, st.probs, st.topk_idx, st.topk_w, p["offsets"],
+                           p["sorted_pair"], p["pair_pos"], st.T, st.E, st.k, W_gu, W_d,
+                           out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream)
+
+
+def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True) -> dict:
+    """Every output and workspace of one forward+backward, allocated once."""
+    P = T * k
+    bf = torch.bfloat16
+    lib = B.lib()
+    d = dict(
+        topk_idx=torch.empty(T, k, dtype=torch.int32, device=device),
+        topk_w=torch.empty(T, k, dtype=torch.float32, device=device),
+        probs=torch.empty(T, E, dtype=torch.float32, device=device),
+        perm=dict(counts=torch.empty(E, dtype=torch.int32, device=device),
+                  offsets=torch.empty(E + 1, dtype=torch.int32, device=device),
+                  sorted_pair=torch.empty(P, dtype=torch.int32, device=device),
+                  pair_pos=torch.empty(P, dtype=torch.int32, device=device),
+                  Xp=torch.empty(P, H, dtype=bf, device=device)),
+        perm_ws=torch.empty(max(lib.moe_permute_workspace_bytes(T, E, k), 1), dtype=torch.uint8, device=device),
+        h=torch.empty(P, I, dtype=bf, device=device),
+        gu=torch.empty(P, 2 * I, dtype=bf, device=device) if save_gu else None,
+        O=torch.empty(P, H, dtype=bf, device=device),
+        Y=torch.empty(T, H, dtype=bf, device=device),
+        grads=dict(dX=torch.empty(T, H, dtype=bf, device=device),
+                   dW_gu=torch.empty(E, 2 * I, H, dtype=bf, device=device),
+                   dW_d=torch.empty(E, H, I, dtype=bf, device=device),
+                   dlogits=torch.empty(T, E, dtype=torch.float32, device=device)),
+        bwd_ws=torch.empty(max(lib.moe_layer_bwd_workspace_bytes(T, E, k, H, I, 0 if save_gu else 1), 1),
+                           dtype=torch.uint8, device=device),
+    )
+    return d

@@ -1,0 +1,74 @@
+"""The C-ABI library builds, loads without a GPU, exports every function the
+header declares, and rejects bad arguments before touching a device."""
+import ctypes
+
+import pytest
+
+from routed_grouped_gemm_router_b200 import binding as B
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    names = B.header_symbols()
+    assert {"moe_route", "moe_permute", "moe_experts_fwd", "moe_combine", "moe_layer_bwd"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libmoe.so does not export {n}"
+
+
+def test_status_strings():
+    assert B.status_str(0) == "MOE_OK"
+    assert B.status_str(1) == "MOE_ERR_INVALID_ARG"
+    assert B.status_str(5) == "MOE_ERR_TIMEOUT"
+    assert B.status_str(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_queries():
+    lib = B.lib()
+    assert lib.moe_permute_workspace_bytes(0, 8, 2) == 0
+    assert lib.moe_permute_workspace_bytes(8192, 128, 8) >= 32 * 128 * 4
+    assert lib.moe_permute_workspace_bytes(4, 2, 3) == 0, "k > E is invalid"
+    P, H, I = 8192 * 8, 2048, 768
+    need = lib.moe_layer_bwd_workspace_bytes(8192, 128, 8, H, I, 0)
+    assert need >= P * (2 * H + 3 * I) * 2
+    assert lib.moe_layer_bwd_workspace_bytes(8192, 128, 8, H, I, 1) >= need + P * 2 * I * 2
+    assert lib.moe_layer_bwd_workspace_bytes(8192, 128, 8, 2047, I, 0) == 0, "H must be a multiple of 8"
+
+
+NULL = None
+
+
+def test_invalid_arguments_rejected_without_device():
+    lib = B.lib()
+    p = ctypes.c_void_p(256)  # aligned dummy address; never dereferenced
+    odd = ctypes.c_void_p(257)
+    # shapes
+    assert lib.moe_route(p, 4, 3, 4, p, p, p, NULL) == 1          # k > E
+    assert lib.moe_route(p, 4, 2000, 4, p, p, p, NULL) == 1       # E > 1024
+    assert lib.moe_route(p, -1, 8, 2, p, p, p, NULL) == 1         # T < 0
+    assert lib.moe_route(p, 1 << 28, 16, 16, p, p, p, NULL) == 1  # T*k >= 2^31
+    # pointers
+    assert lib.moe_route(NULL, 4, 8, 2, p, p, p, NULL) == 1
+    assert lib.moe_route(odd, 4, 8, 2, p, p, p, NULL) == 1
+    assert lib.moe_combine(p, p, 4, 2, 12, p, NULL) == 1          # H not a multiple of 8
+    assert lib.moe_permute(p, 4, 8, 2, NULL, p, p, p, NULL, 0, NULL, p, 4096, NULL) == 1
+    assert lib.moe_permute(p, 4, 8, 2, p, p, p, p, p, 16, NULL, p, 4096, NULL) == 1  # X without Xp
+    # workspace
+    assert lib.moe_permute(p, 4, 8, 2, p, p, p, p, NULL, 0, NULL, p, 0, NULL) == 3
+    need = lib.moe_layer_bwd_workspace_bytes(4, 8, 2, 16, 16, 0)
+    args = [p] * 10 + [4, 8, 2, 16, 16] + [p] * 7
+    assert lib.moe_layer_bwd(*args, p, need - 1, NULL) == 3
+    assert lib.moe_layer_bwd(*([p, p, NULL] + [p] * 7 + [4, 8, 2, 16, 16] + [p] * 7), p, need - 1, NULL) == 3
+
+
+def test_empty_batch_needs_no_device():
+    lib = B.lib()
+    p = ctypes.c_void_p(256)
+    assert lib.moe_route(p, 0, 8, 2, p, p, p, NULL) == 0
+    assert lib.moe_experts_fwd(p, p, p, p, 0, 8, 2, 16, 16, p, p, p, p, p, NULL) == 0
+    assert lib.moe_combine(p, p, 0, 2, 16, p, NULL) == 0
+
+
+def test_profile_names():
+    names = B.profile_kernel_names()
+    assert "gemm_fwd_gate_up" in names and "router_bwd" in names
+    assert len(names) == len(set(names))

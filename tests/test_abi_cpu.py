@@ -55,9 +55,9 @@ def test_invalid_arguments_rejected_without_device():
     # workspace
     assert lib.moe_permute(p, 4, 8, 2, p, p, p, p, NULL, 0, NULL, p, 0, NULL) == 3
     need = lib.moe_layer_bwd_workspace_bytes(4, 8, 2, 16, 16, 0)
-    args = [p] * 10 + [4, 8, 2, 16, 16] + [p] * 7
+    args = [p] * 10 + [4, 8, 2, 16, 16] + [p] * 6
     assert lib.moe_layer_bwd(*args, p, need - 1, NULL) == 3
-    assert lib.moe_layer_bwd(*([p, p, NULL] + [p] * 7 + [4, 8, 2, 16, 16] + [p] * 7), p, need - 1, NULL) == 3
+    assert lib.moe_layer_bwd(*([p, p, NULL] + [p] * 7 + [4, 8, 2, 16, 16] + [p] * 6), p, need - 1, NULL) == 3
 
 
 def test_empty_batch_needs_no_device():

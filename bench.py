@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE expert layer (forward + backward) on B200.
+
+One step = the whole layer: moe_route -> moe_permute -> moe_experts_fwd ->
+moe_combine -> moe_layer_bwd on one synthetic batch already resident in HBM.
+Prints ONE JSON line (rank 0). Default workload: the Qwen3-30B-A3B-shaped
+layer (T=8192, H=2048, E=128, k=8, I=768), forward and backward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+replica on its own batch (weak scaling, no data-path collective); the time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from routed_grouped_gemm_router_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MoE layer fwd/bwd TFLOP/s and tokens/s on 1 B200; % of bf16 tensor peak"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Algorithmic work per launch of each kernel, as a function of the workload:
+# GEMMs in flops (bf16 tensor cores), memory kernels in bytes (HBM).
+def kernel_work(name, wl):
+    T, H, E, k, I, P = wl.T, wl.H, wl.E, wl.k, wl.I, wl.P
+    flops = {
+        "gemm_fwd_gate_up": 4.0 * H * I * P, "gemm_fwd_down": 2.0 * H * I * P,
+        "gemm_recompute_gate_up": 4.0 * H * I * P,
+        "gemm_bwd_dgrad_down": 2.0 * H * I * P, "gemm_bwd_dgrad_gate_up": 4.0 * H * I * P,
+        "gemm_bwd_wgrad_gate_up": 4.0 * H * I * P, "gemm_bwd_wgrad_down": 2.0 * H * I * P,
+    }
+    if name in flops:
+        return "tensor", flops[name]
+    nbytes = {
+        # one read of each source row (L2 serves the k re-reads), one write per pair row
+        "gather_x": T * H * 2 + P * H * 2 + P * 4, "gather_dy": T * H * 2 + P * H * 2 + P * 4,
+        "combine_y": P * H * 2 + T * H * 2 + P * 4, "combine_dx": P * H * 2 + T * H * 2 + P * 4,
+        "route": T * E * 4 * 2 + T * k * 8,
+        "router_bwd": T * E * 4 * 2 + T * k * 12 + P * 4 * ((I + 255) // 256),
+        "permute_count": P * 4, "permute_scan": E * 8, "permute_scatter": P * 12,
+    }
+    return "hbm", float(nbytes.get(name, 0))
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "routed_grouped_gemm_router_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary of the same kernel
+    source; None when there is none or the sources changed since."""
+    sha = kernel_source_sha()
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
+        text = open(p).read()
+        if (re.search(rf"^kernel: {re.escape(kernel)}$", text, re.M)
+                and re.search(rf"^workload: {re.escape(workload)}$", text, re.M)
+                and re.search(rf"^source_sha: {sha}$", text, re.M)):
+            m = re.search(r"^traffic_bytes_per_launch: ([0-9.eE+]+)$", text, re.M)
+            if m:
+                return float(m.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw) if p > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_step(inp_sub, k, backward):
+    from oracle import moe_oracle as orc
+    fwd = orc.layer_forward(inp_sub.logits, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
+    if backward:
+        orc.layer_backward(fwd, inp_sub.dY, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
+
+
+def cpu_sample(inp, wl, target_s):
+    """The first T_s tokens of the batch (all E experts), T_s sized so one
+    oracle fwd+bwd takes about target_s seconds on the host cores."""
+    import copy
+
+    def sub(ts):
+        s = copy.copy(inp)
+        s.X, s.logits = inp.X[:ts].contiguous(), inp.logits[:ts].contiguous()
+        s.dY = inp.dY[:ts].contiguous() if inp.dY is not None else None
+        return s
+
+    ts = min(wl.T, 64)
+    t0 = time.perf_counter()
+    oracle_step(sub(ts), wl.k, wl.backward)
+    dt = time.perf_counter() - t0
+    while ts < wl.T and dt < target_s / 4:
+        ts = min(wl.T, ts * 4)
+        t0 = time.perf_counter()
+        oracle_step(sub(ts), wl.k, wl.backward)
+        dt = time.perf_counter() - t0
+    return sub(ts), ts
+
+
+def step_flops(wl):
+    return wl.flops_fwd() + (wl.flops_bwd() if wl.backward else 0.0)
+
+
+def run_reference(args, wl, rank):
+    """The oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    inp = make_inputs(wl, seed=args.seed)
+    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s)
+    sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
+    for _ in range(args.warmup):
+        oracle_step(sample, wl.k, wl.backward)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sample, wl.k, wl.backward)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = step_flops(sub_wl) / dt / 1e12
+    desc = f"first {ts} of {wl.T} tokens, all {wl.E} experts, {'fwd+bwd' if wl.backward else 'fwd'} in float64"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, args),
+        "tokens_per_s": ts / dt,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, args):
+    return {"workload": f"{wl.name} MoE layer {'fwd+bwd' if wl.backward else 'fwd'}: T={wl.T} H={wl.H} "
+                        f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else ""),
+            "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
+            "l2": "flushed between timed steps (256 MiB write outside the timed events)",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen3-30b-a3b", choices=sorted(WORKLOADS))
+    ap.add_argument("--forward-only", action="store_true")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-target-s", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=4.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.forward_only:
+        wl = type(wl)(wl.name, wl.T, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, False)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import torch.distributed as dist
+    from routed_grouped_gemm_router_b200 import binding as B
+    from routed_grouped_gemm_router_b200 import layer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    # every rank its own batch: seed + rank
+    inp = make_inputs(wl, seed=args.seed + rank, with_dy=wl.backward)
+    X, W_gu, W_d = inp.X.to(dev), inp.W_gu.to(dev), inp.W_d.to(dev)
+    logits = inp.logits.to(dev)
+    dY = inp.dY.to(dev) if wl.backward else None
+    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs)
+        if wl.backward:
+            layer.backward(st, dY, W_gu, W_d, bufs=bufs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = B.last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    B.profile_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    prof = B.profile_read()
+    B.profile_enable(False)
+    status = B.last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timed steps: {B.status_str(status)}")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+
+    # end to end through the public API with host buffers
+    pin = dict(X=inp.X.pin_memory(), logits=inp.logits.pin_memory(),
+               dY=inp.dY.pin_memory() if wl.backward else None)
+    out_h = dict(Y=torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory(),
+                 dX=torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory(),
+                 dlogits=torch.empty(wl.T, wl.E, dtype=torch.float32).pin_memory())
+    h2d = pin["X"].numel() * 2 + pin["logits"].numel() * 4 + (pin["dY"].numel() * 2 if wl.backward else 0)
+    d2h = out_h["Y"].numel() * 2 + ((out_h["dX"].numel() * 2 + out_h["dlogits"].numel() * 4) if wl.backward else 0)
+
+    def e2e_step():
+        X.copy_(pin["X"], non_blocking=True)
+        logits.copy_(pin["logits"], non_blocking=True)
+        if wl.backward:
+            dY.copy_(pin["dY"], non_blocking=True)
+        st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs)
+        out_h["Y"].copy_(st.Y, non_blocking=True)
+        if wl.backward:
+            g = layer.backward(st, dY, W_gu, W_d, bufs=bufs)
+            out_h["dX"].copy_(g["dX"], non_blocking=True)
+            out_h["dlogits"].copy_(g["dlogits"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_evs[i][0].record(stream)
+        e2e_step()
+        e2e_evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+    clocks = sampler.stop() if sampler else None
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = t.tolist()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    flops = step_flops(wl)
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = world * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    peaks, peaks_src = read_peaks()
+
+    # dominant kernel: most device time over the timed region
+    kernels = {}
+    launches = 0
+    for name, (ms, n) in prof.items():
+        kind, work = kernel_work(name, wl)
+        avg_ms = ms / n
+        launches += n
+        rate = work / (avg_ms * 1e-3)
+        kernels[name] = {"ms_per_step": ms / args.steps, "launches": n, "share": ms / total_ms,
+                         "bound": kind,
+                         "achieved": rate / 1e12 if kind == "tensor" else rate / 1e9,
+                         "unit": "TFLOP/s" if kind == "tensor" else "GB/s"}
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0]
+    kind, work = kernel_work(dom, wl)
+    avg_s = prof[dom][0] / prof[dom][1] * 1e-3
+    if kind == "tensor":
+        achieved = work / avg_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_sustained": peaks["bf16_tflops_sustained"],
+                "frac_sustained": achieved / peaks["bf16_tflops_sustained"]}
+    else:
+        achieved = work / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name), "algorithmic_per_launch": work,
+                 "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s)
+        t0 = time.perf_counter()
+        oracle_step(sample, wl.k, wl.backward)
+        dt = time.perf_counter() - t0
+        sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
+        cpu = {"value": step_flops(sub_wl) / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {ts} of {wl.T} tokens, all {wl.E} experts, "
+                         f"{'fwd+bwd' if wl.backward else 'fwd'} in float64, one run of {dt:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+        "config": workload_config(wl, args),
+        "tokens_per_s": world * wl.T * args.steps / (total_ms * 1e-3),
+        "pct_of_bf16_peak": value / world / peaks["bf16_tflops"],
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": launches, "clocks": clocks, "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -131,12 +131,27 @@ __device__ __forceinline__ void store8_bf16(uint16_t* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = o;
 }
 
-__device__ __forceinline__ void load8_bf16(const uint16_t* src, float* v) {
-  const uint4 i = *reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void unpack8(const uint4 i, float* v) {
   v[0] = bf16lo(i.x); v[1] = bf16hi(i.x);
   v[2] = bf16lo(i.y); v[3] = bf16hi(i.y);
   v[4] = bf16lo(i.z); v[5] = bf16hi(i.z);
   v[6] = bf16lo(i.w); v[7] = bf16hi(i.w);
+}
+
+// dgrad-down epilogue operands of one 32-column chunk starting at column i0
+// of row r: g (4 x 16 B), u (4 x 16 B), h (4 x 16 B); zeros past I.
+__device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t r, bool valid, int i0, uint4 (&b)[12]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int i = i0 + 8 * v;
+    if (valid && i < p.I) {
+      b[v] = __ldg(reinterpret_cast<const uint4*>(p.gu + r * (2 * p.I) + i));
+      b[4 + v] = __ldg(reinterpret_cast<const uint4*>(p.gu + r * (2 * p.I) + p.I + i));
+      b[8 + v] = __ldg(reinterpret_cast<const uint4*>(p.h_in + r * p.I + i));
+    } else {
+      b[v] = b[4 + v] = b[8 + v] = make_uint4(0, 0, 0, 0);
+    }
+  }
 }
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
@@ -372,6 +387,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           continue;
         }
       }
+      // dgrad-down: the epilogue reads g, u, h of its row; issue the first
+      // chunk's loads (and the routing weight) before waiting for the
+      // accumulator so their latency hides behind the main loop.
+      uint4 dd_cur[12];
+      int64_t dd_r = 0;
+      bool dd_valid = false;
+      float dd_w = 0.0f;
+      if constexpr (KIND == kBwdDgradDown) {
+        dd_valid = row < ti.rows;
+        dd_r = ti.row0 + row;
+        if (dd_valid) {
+          const int32_t q = p.sorted_pair[dd_r];
+          dd_w = (q >= 0 && q < p.P) ? __ldg(p.topk_w + q) : 0.0f;
+        }
+        dgrad_down_load(p, dd_r, dd_valid, ti.n_blk * kBN, dd_cur);
+      }
       const int acc = tcount & 1;
       if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
         if (lane == 0) report(MOE_ERR_TIMEOUT);
@@ -438,47 +469,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           }
         }
       } else if constexpr (KIND == kBwdDgradDown) {
-        const bool rvalid = row < ti.rows;
-        const int64_t r = ti.row0 + row;
-        float wq = 0.0f;
-        if (rvalid) {
-          const int32_t q = p.sorted_pair[r];
-          wq = (q >= 0 && q < p.P) ? p.topk_w[q] : 0.0f;
-        }
-        float dwp = 0.0f;
         const int I = p.I;
-        for (int c = 0; c < kBN; c += 32) {
+        float dwp = 0.0f;
+#pragma unroll
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int i0 = ti.n_blk * kBN + ch * 32;
+          uint4 nxt[12];
+          if (ch + 1 < kBN / 32) dgrad_down_load(p, dd_r, dd_valid, i0 + 32, nxt);
           uint32_t a[32];
-          tmem_ld_32x32b_x32(taddr + c, a);
+          tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
-          const int i0 = ti.n_blk * kBN + c;
-          if (rvalid && i0 < I) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int i = i0 + 8 * v;
-              if (i < I) {
-                float gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
-                load8_bf16(p.gu + r * (2 * I) + i, gv);
-                load8_bf16(p.gu + r * (2 * I) + I + i, uv);
-                load8_bf16(p.h_in + r * I + i, hv);
+          for (int v = 0; v < 4; ++v) {
+            const int i = i0 + 8 * v;
+            if (dd_valid && i < I) {
+              float gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
+              unpack8(dd_cur[v], gv);
+              unpack8(dd_cur[4 + v], uv);
+              unpack8(dd_cur[8 + v], hv);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const float dhp = __uint_as_float(a[8 * v + j]);
-                  dwp += dhp * hv[j];
-                  const float dh = wq * dhp;
-                  const float s = sigmoid_f(gv[j]);
-                  du[j] = dh * gv[j] * s;
-                  dg[j] = dh * uv[j] * s * (1.0f + gv[j] * (1.0f - s));
-                  hw[j] = wq * hv[j];
-                }
-                store8_bf16(p.out + r * p.out_ld + i, dg);
-                store8_bf16(p.out + r * p.out_ld + I + i, du);
-                store8_bf16(p.hw_out + r * I + i, hw);
+              for (int j = 0; j < 8; ++j) {
+                const float dhp = __uint_as_float(a[8 * v + j]);
+                dwp += dhp * hv[j];
+                const float dh = dd_w * dhp;
+                const float sg = sigmoid_f(gv[j]);
+                du[j] = dh * gv[j] * sg;
+                dg[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));
+                hw[j] = dd_w * hv[j];
               }
+              store8_bf16(p.out + dd_r * p.out_ld + i, dg);
+              store8_bf16(p.out + dd_r * p.out_ld + I + i, du);
+              store8_bf16(p.hw_out + dd_r * I + i, hw);
             }
           }
+          if (ch + 1 < kBN / 32) {
+#pragma unroll
+            for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
+          }
         }
-        if (rvalid) p.dw_part[r * p.n_tiles + ti.n_blk] = dwp;
+        if (dd_valid) p.dw_part[dd_r * p.n_tiles + ti.n_blk] = dwp;
       } else {  // wgrad
         const int m = ti.m_blk * kBM + row;
         const bool mvalid = m < p.M;

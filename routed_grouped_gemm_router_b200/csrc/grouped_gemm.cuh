@@ -49,6 +49,11 @@ constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
 constexpr int kNumBarriers = 2 * kStages + 5;
+// Epilogue staging: per epilogue warp 32 rows x 32 fp32 with a 36-float row
+// stride, so both the row-wise 16-byte writes (8 lanes = 8 rows per phase)
+// and the transposed 16-byte reads (8 lanes = 8 rows per phase) hit 8
+// distinct bank groups.
+constexpr int kStageStride = 36;
 
 struct GemmParams {
   CUtensorMap tmA;
@@ -76,7 +81,7 @@ struct GemmParams {
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
   return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes + kNumBarriers * 8 + 16 +
-         2 * static_cast<size_t>(E + 1) * 4;
+         2 * static_cast<size_t>(E + 1) * 4 + 16 + 4 * 32 * kStageStride * 4;
 }
 
 struct TileInfo {
@@ -138,18 +143,64 @@ __device__ __forceinline__ void unpack8(const uint4 i, float* v) {
   v[6] = bf16lo(i.w); v[7] = bf16hi(i.w);
 }
 
-// dgrad-down epilogue operands of one 32-column chunk starting at column i0
-// of row r: g (4 x 16 B), u (4 x 16 B), h (4 x 16 B); zeros past I.
-__device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t r, bool valid, int i0, uint4 (&b)[12]) {
+__device__ __forceinline__ void stage_row(float* stg, int lane, const uint32_t (&v)[32]) {
+  float* rp = stg + lane * kStageStride;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const int i = i0 + 8 * v;
-    if (valid && i < p.I) {
-      b[v] = __ldg(reinterpret_cast<const uint4*>(p.gu + r * (2 * p.I) + i));
-      b[4 + v] = __ldg(reinterpret_cast<const uint4*>(p.gu + r * (2 * p.I) + p.I + i));
-      b[8 + v] = __ldg(reinterpret_cast<const uint4*>(p.h_in + r * p.I + i));
+  for (int m = 0; m < 8; ++m)
+    *reinterpret_cast<uint4*>(rp + 4 * m) = make_uint4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+}
+
+__device__ __forceinline__ void stage_row(float* stg, int lane, const float (&v)[32]) {
+  float* rp = stg + lane * kStageStride;
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+    *reinterpret_cast<float4*>(rp + 4 * m) = make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+}
+
+// 8 consecutive staged values of row r starting at column 8*q.
+__device__ __forceinline__ void read_transposed(const float* stg, int r, int q, float (&o)[8]) {
+  const float* rp = stg + r * kStageStride + q * 8;
+  const float4 a = *reinterpret_cast<const float4*>(rp);
+  const float4 b = *reinterpret_cast<const float4*>(rp + 4);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
+// Stores one 32-column chunk (row domain values v, thread = row) as bf16 to
+// base[(row0 + r) * ld + col0 + c] for the warp's valid rows and c < ncols.
+__device__ __forceinline__ void emit_chunk(float* stg, const float (&v)[32], uint16_t* base, int64_t row0,
+                                           int64_t ld, int col0, int ncols, int wrows, int tr_row, int tr_q,
+                                           int lane) {
+  stage_row(stg, lane, v);
+  __syncwarp();
+  const int col = col0 + tr_q * 8;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + tr_row;
+    if (r < wrows && col < ncols) {
+      float o[8];
+      read_transposed(stg, r, tr_q, o);
+      store8_bf16(base + (row0 + r) * ld + col, o);
+    }
+  }
+  __syncwarp();
+}
+
+// dgrad-down epilogue operands in the transposed domain: for rows 8*i + tr_row
+// of the warp, 8 columns from `col`: g, u and h (16 bytes each); zeros for
+// rows or columns that do not exist.
+__device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t wrow0, int wrows, int col, int tr_row,
+                                                uint4 (&b)[12]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + tr_row;
+    if (r < wrows && col < p.I) {
+      const int64_t gr = wrow0 + r;
+      b[3 * i] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + col));
+      b[3 * i + 1] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + p.I + col));
+      b[3 * i + 2] = __ldg(reinterpret_cast<const uint4*>(p.h_in + gr * p.I + col));
     } else {
-      b[v] = b[4 + v] = b[8 + v] = make_uint4(0, 0, 0, 0);
+      b[3 * i] = b[3 * i + 1] = b[3 * i + 2] = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -182,6 +233,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
   int* s_tstart = s_off + (p.E + 1);
+  float* s_stage = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -371,38 +423,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     warp_wait(drain_bar, 0);
   } else {
     // ------------------------------------------------------- epilogue
-    const int sub = warp & 3;           // TMEM sub-partition this warp may access
-    const int row = sub * 32 + lane;    // accumulator row (TMEM lane)
+    // Thread (warp w, lane l) reads TMEM lane 32*(w%4)+l: one accumulator row
+    // ("row domain"). Every 32-column chunk is staged through the warp's own
+    // shared buffer and read back transposed ("transposed domain"): lane l
+    // then owns rows 8*i + (l%8), i = 0..3, and columns 8*(l/8)..+7 of the
+    // chunk, so each global load/store instruction covers 8 rows x 64
+    // contiguous bytes instead of 32 rows x 16 bytes.
+    const int sub = warp & 3;
+    const int tr_row = lane & 7;
+    const int tr_q = lane >> 3;
+    float* stg = s_stage + (warp - 2) * 32 * kStageStride;
     int tcount = 0;
     for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+      // valid rows of this warp's 32 (rows past the segment / past M are skipped)
+      const int tile_rows = kWgrad ? min(kBM, p.M - ti.m_blk * kBM) : ti.rows;
+      const int wrows = max(0, min(32, tile_rows - sub * 32));
+      // first output row of this warp: permuted row (row-grouped) or dW row (wgrad)
+      const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + sub * 32
+                                   : static_cast<int64_t>(ti.row0) + sub * 32;
+      uint16_t* out_base = kWgrad ? p.out + ti.e * p.out_expert_stride : p.out;
       if constexpr (kWgrad) {
-        if (ti.num_kb == 0) {
-          const int m = ti.m_blk * kBM + row;
-          if (m < p.M) {
-            uint16_t* dst = p.out + ti.e * p.out_expert_stride + static_cast<int64_t>(m) * p.out_ld;
-            for (int c = ti.n_blk * kBN; c < min(p.N, ti.n_blk * kBN + kBN); c += 8)
-              *reinterpret_cast<uint4*>(dst + c) = make_uint4(0, 0, 0, 0);
+        if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero
+          for (int c = 0; c < kBN; c += 32) {
+            const int col = ti.n_blk * kBN + c + tr_q * 8;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = i * 8 + tr_row;
+              if (r < wrows && col < p.N)
+                *reinterpret_cast<uint4*>(out_base + (wrow0 + r) * p.out_ld + col) = make_uint4(0, 0, 0, 0);
+            }
           }
           continue;
         }
       }
-      // dgrad-down: the epilogue reads g, u, h of its row; issue the first
-      // chunk's loads (and the routing weight) before waiting for the
-      // accumulator so their latency hides behind the main loop.
-      uint4 dd_cur[12];
-      int64_t dd_r = 0;
-      bool dd_valid = false;
-      float dd_w = 0.0f;
-      if constexpr (KIND == kBwdDgradDown) {
-        dd_valid = row < ti.rows;
-        dd_r = ti.row0 + row;
-        if (dd_valid) {
-          const int32_t q = p.sorted_pair[dd_r];
-          dd_w = (q >= 0 && q < p.P) ? __ldg(p.topk_w + q) : 0.0f;
+      // per-row routing weight, row domain (lane = row within the warp)
+      float wq = 1.0f;
+      if constexpr (KIND == kFwdDown || KIND == kBwdDgradDown) {
+        if (lane < wrows && p.topk_w != nullptr) {
+          const int32_t q = p.sorted_pair[wrow0 + lane];
+          wq = (q >= 0 && q < p.P) ? __ldg(p.topk_w + q) : 0.0f;
         }
-        dgrad_down_load(p, dd_r, dd_valid, ti.n_blk * kBN, dd_cur);
       }
+      // dgrad-down: issue the first chunk's g/u/h loads before the wait so
+      // their latency hides behind the main loop
+      uint4 dd_cur[12];
+      if constexpr (KIND == kBwdDgradDown)
+        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + tr_q * 8, tr_row, dd_cur);
+
       const int acc = tcount & 1;
       if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
         if (lane == 0) report(MOE_ERR_TIMEOUT);
@@ -413,121 +481,94 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(sub * 32) << 16);
 
       if constexpr (KIND == kFwdGateUp) {
-        const bool rvalid = row < ti.rows;
-        const int64_t r = ti.row0 + row;
-        for (int c = 0; c < 128; c += 32) {
+        const int I = p.I;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
           uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(taddr + c, g);
-          tmem_ld_32x32b_x32(taddr + 128 + c, u);
+          tmem_ld_32x32b_x32(taddr + ch * 32, g);
+          tmem_ld_32x32b_x32(taddr + 128 + ch * 32, u);
           tmem_ld_wait();
-          const int i0 = ti.n_blk * 128 + c;
-          if (rvalid && i0 < p.I) {
+          const int col0 = ti.n_blk * 128 + ch * 32;
+          if (col0 >= I) continue;  // warp-uniform
+          float v[32];
+          if (p.out != nullptr) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (i0 + 8 * v < p.I) {
-                float hv[8], gv[8], uv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  gv[j] = __uint_as_float(g[8 * v + j]);
-                  uv[j] = __uint_as_float(u[8 * v + j]);
-                  hv[j] = silu_f(gv[j]) * uv[j];
-                }
-                if (p.out != nullptr) store8_bf16(p.out + r * p.out_ld + i0 + 8 * v, hv);
-                if (p.gu != nullptr) {
-                  store8_bf16(p.gu + r * (2 * p.I) + i0 + 8 * v, gv);
-                  store8_bf16(p.gu + r * (2 * p.I) + p.I + i0 + 8 * v, uv);
-                }
-              }
-            }
+            for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+            emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, I, wrows, tr_row, tr_q, lane);
           }
-        }
-      } else if constexpr (KIND == kFwdDown || KIND == kBwdDgradGateUp) {
-        const bool rvalid = row < ti.rows;
-        const int64_t r = ti.row0 + row;
-        float wq = 1.0f;
-        if constexpr (KIND == kFwdDown) {
-          if (rvalid && p.topk_w != nullptr) {
-            const int32_t q = p.sorted_pair[r];
-            wq = (q >= 0 && q < p.P) ? p.topk_w[q] : 0.0f;
-          }
-        }
-        for (int c = 0; c < kBN; c += 32) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(taddr + c, a);
-          tmem_ld_wait();
-          const int n0 = ti.n_blk * kBN + c;
-          if (rvalid && n0 < p.N) {
+          if (p.gu != nullptr) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (n0 + 8 * v < p.N) {
-                float o[8];
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(g[j]);
+            emit_chunk(stg, v, p.gu, wrow0, 2 * I, col0, I, wrows, tr_row, tr_q, lane);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = wq * __uint_as_float(a[8 * v + j]);
-                store8_bf16(p.out + r * p.out_ld + n0 + 8 * v, o);
-              }
-            }
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
+            emit_chunk(stg, v, p.gu + I, wrow0, 2 * I, col0, I, wrows, tr_row, tr_q, lane);
           }
         }
       } else if constexpr (KIND == kBwdDgradDown) {
         const int I = p.I;
-        float dwp = 0.0f;
+        float dwp[4] = {0.f, 0.f, 0.f, 0.f};
+        float wrow[4];
 #pragma unroll
+        for (int i = 0; i < 4; ++i) wrow[i] = __shfl_sync(0xffffffffu, wq, i * 8 + tr_row);
+#pragma unroll 1
         for (int ch = 0; ch < kBN / 32; ++ch) {
-          const int i0 = ti.n_blk * kBN + ch * 32;
+          const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
           uint4 nxt[12];
-          if (ch + 1 < kBN / 32) dgrad_down_load(p, dd_r, dd_valid, i0 + 32, nxt);
+          if (ch + 1 < kBN / 32) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
           uint32_t a[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
+          stage_row(stg, lane, a);
+          __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int i = i0 + 8 * v;
-            if (dd_valid && i < I) {
-              float gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
-              unpack8(dd_cur[v], gv);
-              unpack8(dd_cur[4 + v], uv);
-              unpack8(dd_cur[8 + v], hv);
+          for (int i = 0; i < 4; ++i) {
+            const int r = i * 8 + tr_row;
+            if (r < wrows && col < I) {
+              float dhp[8], gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
+              read_transposed(stg, r, tr_q, dhp);
+              unpack8(dd_cur[3 * i], gv);
+              unpack8(dd_cur[3 * i + 1], uv);
+              unpack8(dd_cur[3 * i + 2], hv);
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const float dhp = __uint_as_float(a[8 * v + j]);
-                dwp += dhp * hv[j];
-                const float dh = dd_w * dhp;
+                dwp[i] += dhp[j] * hv[j];
+                const float dh = wrow[i] * dhp[j];
                 const float sg = sigmoid_f(gv[j]);
                 du[j] = dh * gv[j] * sg;
                 dg[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));
-                hw[j] = dd_w * hv[j];
+                hw[j] = wrow[i] * hv[j];
               }
-              store8_bf16(p.out + dd_r * p.out_ld + i, dg);
-              store8_bf16(p.out + dd_r * p.out_ld + I + i, du);
-              store8_bf16(p.hw_out + dd_r * I + i, hw);
+              const int64_t gr = wrow0 + r;
+              store8_bf16(p.out + gr * p.out_ld + col, dg);
+              store8_bf16(p.out + gr * p.out_ld + I + col, du);
+              store8_bf16(p.hw_out + gr * I + col, hw);
             }
           }
-          if (ch + 1 < kBN / 32) {
+          __syncwarp();
 #pragma unroll
-            for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
-          }
+          for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
         }
-        if (dd_valid) p.dw_part[dd_r * p.n_tiles + ti.n_blk] = dwp;
-      } else {  // wgrad
-        const int m = ti.m_blk * kBM + row;
-        const bool mvalid = m < p.M;
-        uint16_t* dst = p.out + ti.e * p.out_expert_stride + static_cast<int64_t>(m) * p.out_ld;
-        for (int c = 0; c < kBN; c += 32) {
+        // each row's partial dot product is spread over the 4 lanes with the same l%8
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 8);
+          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 16);
+          const int r = i * 8 + tr_row;
+          if (tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * p.n_tiles + ti.n_blk] = dwp[i];
+        }
+      } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
+#pragma unroll 1
+        for (int ch = 0; ch < kBN / 32; ++ch) {
           uint32_t a[32];
-          tmem_ld_32x32b_x32(taddr + c, a);
+          tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
-          const int n0 = ti.n_blk * kBN + c;
-          if (mvalid && n0 < p.N) {
+          const int col0 = ti.n_blk * kBN + ch * 32;
+          if (col0 >= p.N) continue;  // warp-uniform
+          float v[32];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (n0 + 8 * v < p.N) {
-                float o[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(a[8 * v + j]);
-                store8_bf16(dst + n0 + 8 * v, o);
-              }
-            }
-          }
+          for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a[j]);
+          emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane);
         }
       }
       tc_fence_before();

@@ -6,27 +6,32 @@
 // routing-weight multiply fused after the GEMM ("fuse_mul_post").
 //
 // B200 design (not a translation of the Triton kernels):
-//  * one CTA per SM, 6 warps: warp 0 issues TMA loads, warp 1 issues tcgen05
-//    MMAs (and owns the TMEM allocation), warps 2-5 run the epilogue;
-//  * 128 x 256 output tiles, K staged 64 at a time through a 4-deep ring of
-//    128-byte-swizzled shared-memory tiles fed by TMA, synchronised with
-//    mbarriers (TMA -> MMA "full", MMA commit -> TMA "empty");
-//  * the fp32 accumulator lives in TMEM, double-buffered (2 x 256 columns),
-//    so the epilogue of tile i overlaps the main loop of tile i+1;
+//  * CTA pairs (clusters of 2 on one TPC) run tcgen05 MMAs of 256 x 256 x 16:
+//    each CTA stages its own 128 rows of A and its half (128 rows) of B, the
+//    even CTA issues the MMA for both, and each CTA's TMEM receives its 128
+//    accumulator rows. Per CTA a 64-deep K step is 32 KiB, so a 6-deep
+//    TMA ring fits in shared memory;
+//  * 6 warps per CTA: warp 0 issues TMA loads, warp 1 issues MMAs (even CTA)
+//    and owns the TMEM allocation, warps 2-5 run the epilogue;
+//  * both CTAs' loads complete on the even CTA's "full" mbarrier; the MMA
+//    warp's commits release the "empty" barriers of both CTAs; the fp32
+//    accumulator is double-buffered in TMEM (2 x 256 columns) so the
+//    epilogue of tile i overlaps the main loop of tile i+1;
 //  * the tile list is built on the device from the per-expert offsets, so the
 //    host never learns the counts and experts without rows cost nothing.
 //
 // Variants (all D = A * B^T with bf16 operands and fp32 accumulation):
-//  FwdGateUp   A = Xp[P,H] (K-major), B = W_gu[e] gate rows and up rows
-//              interleaved per tile (128 + 128), epilogue h = silu(g) * u.
+//  FwdGateUp   A = Xp[P,H] (K-major), B = gate rows (even CTA) and up rows
+//              (odd CTA) of W_gu[e]; epilogue h = silu(g) * u.
 //  FwdDown     A = h[P,I], B = W_d[e][H,I], epilogue O = w_q * acc.
 //  BwdDgradDown   A = dYp[P,H], B = W_d[e] read MN-major ([H,I] as K x N);
 //              epilogue: partial dw = <acc, h>, dh = w_q*acc, SwiGLU backward
 //              -> dGU = [dg | du], and hw = w_q * h for the down wgrad.
 //  BwdDgradGateUp A = dGU[P,2I], B = W_gu[e] MN-major ([2I,H] as K x N) -> dXp.
 //  BwdWgrad    per expert dW[e] = A^T B with the expert's rows as K; both
-//              operands MN-major; the last K block of a segment is clipped
-//              by zeroing the rows past the segment in shared memory.
+//              operands MN-major, loaded through per-expert tensor maps whose
+//              row extent ends at the segment end, so TMA reads the rows of
+//              the next expert as zeros.
 #pragma once
 #include <cuda.h>
 
@@ -37,13 +42,15 @@ namespace moe {
 
 enum GemmKind : int { kFwdGateUp = 0, kFwdDown = 1, kBwdDgradDown = 2, kBwdDgradGateUp = 3, kBwdWgrad = 4 };
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBM = 256;        // rows of a pair tile
+constexpr int kBMc = 128;       // rows per CTA
+constexpr int kBN = 256;        // columns of a tile (accumulator columns per CTA)
+constexpr int kBNc = 128;       // B rows (N) staged per CTA
 constexpr int kBK = 64;
 constexpr int kUmmaK = 16;
-constexpr int kStages = 4;
-constexpr int kATileBytes = kBM * kBK * 2;  // 16 KiB
-constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KiB
+constexpr int kStages = 6;
+constexpr int kATileBytes = kBMc * kBK * 2;  // 16 KiB
+constexpr int kBTileBytes = kBNc * kBK * 2;  // 16 KiB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;
@@ -58,6 +65,7 @@ constexpr int kStageStride = 36;
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  const CUtensorMap* expert_maps;  // wgrad: [2][E] maps (A then B) clipped at each segment end
   const int32_t* offsets;      // [E+1] expert segment bounds in the permuted rows
   const int32_t* sorted_pair;  // [P]
   const float* topk_w;         // [P] routing weight per pair id (NULL: 1)
@@ -86,8 +94,8 @@ __host__ __device__ inline size_t gemm_smem_bytes(int E) {
 
 struct TileInfo {
   int e, m_blk, n_blk;
-  int row0;     // first permuted row (row-grouped) / first K row (wgrad)
-  int rows;     // valid rows in the tile (row-grouped) / rows of the segment (wgrad)
+  int row0;     // first permuted row of the pair tile (row-grouped) / first K row (wgrad)
+  int rows;     // rows of the segment from row0 on (row-grouped) / rows of the segment (wgrad)
   int num_kb;   // K blocks
 };
 
@@ -115,7 +123,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.m_blk = local / p.n_tiles;
     ti.n_blk = local - ti.m_blk * p.n_tiles;
     ti.row0 = s_off[lo] + ti.m_blk * kBM;
-    ti.rows = min(kBM, s_off[lo + 1] - ti.row0);
+    ti.rows = s_off[lo + 1] - ti.row0;
     ti.num_kb = (p.K + kBK - 1) / kBK;
   }
   return ti;
@@ -209,7 +217,8 @@ __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
 template <int KIND>
-__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool kWgrad = (KIND == kBwdWgrad);
   constexpr bool kAMN = kWgrad;
   constexpr bool kBMN = (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || kWgrad);
@@ -224,10 +233,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kATileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* full_bar = bars;
-  uint64_t* empty_bar = bars + kStages;
-  uint64_t* tfull_bar = bars + 2 * kStages;
-  uint64_t* tempty_bar = bars + 2 * kStages + 2;
+  uint64_t* full_bar = bars;                 // even CTA: both CTAs' TMA bytes of a stage
+  uint64_t* empty_bar = bars + kStages;      // each CTA: its stage may be refilled
+  uint64_t* tfull_bar = bars + 2 * kStages;  // each CTA: accumulator buffer ready
+  uint64_t* tempty_bar = bars + 2 * kStages + 2;  // even CTA: both epilogues done with a buffer
   uint64_t* drain_bar = bars + 2 * kStages + 4;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBarriers);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
@@ -237,6 +246,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
 
   // ------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -246,7 +258,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], 2 * 128);
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -257,13 +269,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(s_tmem, kTmemCols);
+    tmem_relinquish_pair();
   }
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
   __syncthreads();
   if (warp == 0 && !kWgrad) {
-    // tiles of expert e = ceil(rows_e / BM) * n_tiles; exclusive prefix over experts
+    // pair tiles of expert e = ceil(rows_e / 256) * n_tiles; exclusive prefix over experts
     const int per = (p.E + 31) / 32;
     const int e0 = lane * per;
     int local = 0;
@@ -284,6 +296,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int total_tiles = kWgrad ? p.E * p.m_tiles * p.n_tiles : s_tstart[p.E];
@@ -294,42 +307,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
+      for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
         const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        const CUtensorMap* mapA = &p.tmA;
+        const CUtensorMap* mapB = &p.tmB;
+        if constexpr (kWgrad) {
+          if (ti.num_kb == 0) continue;
+          mapA = p.expert_maps + ti.e;
+          mapB = p.expert_maps + p.E + ti.e;
+          tensormap_acquire(mapA);
+          tensormap_acquire(mapB);
+        }
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             report(MOE_ERR_TIMEOUT);
             *s_abort = 1;
             break;
           }
-          mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
           const int kx = kb * kBK;
           if constexpr (KIND == kFwdGateUp) {
-            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
-            const int gate_row = ti.e * p.b_rows + ti.n_blk * 128;
-            tma_load_2d(b_dst, &p.tmB, &full_bar[stage], kx, gate_row);
-            tma_load_2d(b_dst + 16384, &p.tmB, &full_bar[stage], kx, gate_row + p.I);
+            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
+            // even CTA: the tile's 128 gate rows; odd CTA: the matching up rows
+            tma_load_2d_pair(b_dst, mapB, fb, kx, ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * p.I);
           } else if constexpr (KIND == kFwdDown) {
-            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
-            const int brow = ti.e * p.b_rows + ti.n_blk * kBN;
-            tma_load_2d(b_dst, &p.tmB, &full_bar[stage], kx, brow);
-            tma_load_2d(b_dst + 16384, &p.tmB, &full_bar[stage], kx, brow + 128);
+            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
+            tma_load_2d_pair(b_dst, mapB, fb, kx, ti.e * p.b_rows + ti.n_blk * kBN + static_cast<int>(rank) * kBNc);
           } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
-            tma_load_2d(a_dst, &p.tmA, &full_bar[stage], kx, ti.row0);
+            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
             const int krow = ti.e * p.b_rows + kx;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tma_load_2d(b_dst + c * 8192, &p.tmB, &full_bar[stage], ti.n_blk * kBN + 64 * c, krow);
+            const int n0 = ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
+            tma_load_2d_pair(b_dst, mapB, fb, n0, krow);
+            tma_load_2d_pair(b_dst + 8192, mapB, fb, n0 + 64, krow);
           } else {  // wgrad: K rows are the expert's permuted rows
             const int krow = ti.row0 + kx;
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_2d(a_dst + c * 8192, &p.tmA, &full_bar[stage], ti.m_blk * kBM + 64 * c, krow);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tma_load_2d(b_dst + c * 8192, &p.tmB, &full_bar[stage], ti.n_blk * kBN + 64 * c, krow);
+            const int m0 = ti.m_blk * kBM + static_cast<int>(rank) * kBMc;
+            const int n0 = ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
+            tma_load_2d_pair(a_dst, mapA, fb, m0, krow);
+            tma_load_2d_pair(a_dst + 8192, mapA, fb, m0 + 64, krow);
+            tma_load_2d_pair(b_dst, mapB, fb, n0, krow);
+            tma_load_2d_pair(b_dst + 8192, mapB, fb, n0 + 64, krow);
           }
           ++issued;
           if (++stage == kStages) {
@@ -338,89 +358,81 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           }
         }
       }
-      // Let every load still in flight land before the block may exit
-      // (immediate in normal operation: the consumer has waited on them).
-      const int inflight = issued < kStages ? issued : kStages;
-      for (int i = 0; i < inflight; ++i) {
-        if (--stage < 0) {
-          stage = kStages - 1;
-          phase ^= 1u;
+      // The even CTA's full barriers count both CTAs' bytes: waiting on the
+      // last phases there means no load of the pair is still in flight when
+      // the pair leaves (immediate in normal operation).
+      if (rank == 0) {
+        const int inflight = issued < kStages ? issued : kStages;
+        for (int i = 0; i < inflight; ++i) {
+          if (--stage < 0) {
+            stage = kStages - 1;
+            phase ^= 1u;
+          }
+          mbar_wait(&full_bar[stage], phase);
         }
-        mbar_wait(&full_bar[stage], phase);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int tcount = 0;
-    for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
-      const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
-      if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogue writes zeros
-      const int acc = tcount & 1;
-      if (!warp_wait(&tempty_bar[acc], ((tcount >> 1) & 1) ^ 1u)) {
-        if (lane == 0) report(MOE_ERR_TIMEOUT);
-        *s_abort = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-      bool ok = true;
-      for (int kb = 0; kb < ti.num_kb; ++kb) {
-        if (!warp_wait(&full_bar[stage], phase)) {
-          ok = false;
+    // ------------------------------------------------------- MMA issuer (even CTA)
+    if (rank == 0) {
+      const uint32_t peer_empty0 = mapa_shared(smem_u32(&empty_bar[0]), 1);
+      const uint32_t peer_tfull0 = mapa_shared(smem_u32(&tfull_bar[0]), 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      int tcount = 0;
+      for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
+        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogues write zeros
+        const int acc = tcount & 1;
+        if (!warp_wait(&tempty_bar[acc], ((tcount >> 1) & 1) ^ 1u)) {
+          if (lane == 0) report(MOE_ERR_TIMEOUT);
+          *s_abort = 1;
           break;
         }
         tc_fence_after();
-        if constexpr (kWgrad) {
-          const int valid = ti.rows - kb * kBK;
-          if (valid < kBK) {
-            // rows past the segment belong to the next expert: zero them in
-            // both 64-column chunks of the A tile (whole 128-byte rows, so the
-            // swizzle does not matter)
-            uint8_t* a_tile = sA + stage * kATileBytes;
-            const int nrows = kBK - valid;
-            for (int i = lane; i < 2 * nrows * 8; i += 32) {
-              const int chunk = i / (nrows * 8);
-              const int rem = i - chunk * nrows * 8;
-              const int r = valid + rem / 8;
-              const int v16 = rem & 7;
-              *reinterpret_cast<uint4*>(a_tile + chunk * 8192 + r * 128 + v16 * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        bool ok = true;
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!warp_wait(&full_bar[stage], phase)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(sA + stage * kATileBytes);
+            const uint32_t b_addr = smem_u32(sB + stage * kBTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+              const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
+              const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
+              umma_bf16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(smem_u32(&empty_bar[stage]));
+            umma_commit_pair(peer_empty0 + stage * 8);
+          }
+          __syncwarp();
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) {
+          if (lane == 0) report(MOE_ERR_TIMEOUT);
+          *s_abort = 1;
+          break;
         }
         if (lane == 0) {
-          const uint32_t a_addr = smem_u32(sA + stage * kATileBytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
-            const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty_bar[stage]);
+          umma_commit_pair(smem_u32(&tfull_bar[acc]));
+          umma_commit_pair(peer_tfull0 + acc * 8);
         }
         __syncwarp();
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        ++tcount;
       }
-      if (!ok) {
-        if (lane == 0) report(MOE_ERR_TIMEOUT);
-        *s_abort = 1;
-        break;
-      }
-      if (lane == 0) umma_commit(&tfull_bar[acc]);
+      // all MMAs of the pair must finish before TMEM is released
+      if (lane == 0) umma_commit_pair(smem_u32(drain_bar));
       __syncwarp();
-      ++tcount;
+      warp_wait(drain_bar, 0);
     }
-    // all MMAs issued by this warp must finish before TMEM is released
-    if (lane == 0) umma_commit(drain_bar);
-    __syncwarp();
-    warp_wait(drain_bar, 0);
   } else {
     // ------------------------------------------------------- epilogue
     // Thread (warp w, lane l) reads TMEM lane 32*(w%4)+l: one accumulator row
@@ -433,15 +445,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     const int tr_row = lane & 7;
     const int tr_q = lane >> 3;
     float* stg = s_stage + (warp - 2) * 32 * kStageStride;
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     int tcount = 0;
-    for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x) {
+    for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
-      // valid rows of this warp's 32 (rows past the segment / past M are skipped)
-      const int tile_rows = kWgrad ? min(kBM, p.M - ti.m_blk * kBM) : ti.rows;
-      const int wrows = max(0, min(32, tile_rows - sub * 32));
+      // this CTA's 128 rows of the pair tile, this warp's 32 of them
+      const int cta_row0 = static_cast<int>(rank) * kBMc + sub * 32;
+      const int tile_rows = kWgrad ? p.M - ti.m_blk * kBM : ti.rows;
+      const int wrows = max(0, min(32, tile_rows - cta_row0));
       // first output row of this warp: permuted row (row-grouped) or dW row (wgrad)
-      const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + sub * 32
-                                   : static_cast<int64_t>(ti.row0) + sub * 32;
+      const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + cta_row0
+                                   : static_cast<int64_t>(ti.row0) + cta_row0;
       uint16_t* out_base = kWgrad ? p.out + ti.e * p.out_expert_stride : p.out;
       if constexpr (kWgrad) {
         if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero
@@ -479,7 +493,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(sub * 32) << 16);
-
       if constexpr (KIND == kFwdGateUp) {
         const int I = p.I;
 #pragma unroll 1
@@ -572,7 +585,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty_bar[acc]);
+      mbar_arrive_cluster(leader_tempty0 + acc * 8);
       ++tcount;
     }
   }
@@ -580,10 +593,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   // ------------------------------------------------------------- tear-down
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the pair's MMAs, loads and TMEM reads are all finished
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+}
+
+// Writes, for each expert e, copies of the A and B tensor maps of the weight
+// gradient whose row extent ends at offsets[e+1] (the end of the expert's
+// segment): out[e] for A, out[E + e] for B. One warp per map.
+__global__ void __launch_bounds__(256) build_expert_maps_kernel(const __grid_constant__ CUtensorMap base_a,
+                                                                const __grid_constant__ CUtensorMap base_b,
+                                                                const int32_t* __restrict__ offsets, int E,
+                                                                CUtensorMap* __restrict__ out) {
+  __shared__ alignas(128) CUtensorMap s_map[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 8 + warp;
+  if (m >= 2 * E) return;  // warp-uniform
+  const int e = m < E ? m : m - E;
+  const CUtensorMap& src = m < E ? base_a : base_b;
+  if (lane < 8)
+    reinterpret_cast<uint4*>(&s_map[warp])[lane] = reinterpret_cast<const uint4*>(&src)[lane];
+  __syncwarp();
+  if (lane == 0) {
+    const int end = offsets[e + 1];
+    tensormap_set_rows(&s_map[warp], static_cast<uint32_t>(end > 0 ? end : 1));
+  }
+  __syncwarp();
+  tensormap_copy_release(out + m, &s_map[warp]);
 }
 
 }  // namespace moe

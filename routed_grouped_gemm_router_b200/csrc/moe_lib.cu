@@ -180,11 +180,15 @@ int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
 
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
-// Persistent grid for the row-grouped GEMMs: at most one CTA per SM and no
-// more than the largest possible tile count.
+// Persistent grid for the GEMMs: CTA pairs, at most one CTA per SM and no
+// more pairs than tiles. Always even (clusters of two).
+inline int pair_grid(int64_t tiles, int num_sms) {
+  const int64_t pairs = num_sms / 2;
+  const int64_t n = tiles < pairs ? tiles : pairs;
+  return static_cast<int>(2 * (n > 0 ? n : 1));
+}
 inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
-  const int64_t bound = (static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles;
-  return static_cast<int>(bound < num_sms ? bound : num_sms);
+  return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
 }
 
 GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
@@ -202,10 +206,9 @@ bool shape_ok(int T, int E, int k) {
 bool dims_ok(int H) { return H > 0 && H % 8 == 0; }
 
 struct BwdLayout {
-  size_t dYp, dGU, hw, dXp, dw_part, gu, total;
+  size_t dYp, dGU, hw, dXp, dw_part, maps, gu, total;
 };
 BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
-  (void)E;
   const size_t P = static_cast<size_t>(T) * k;
   BwdLayout L;
   size_t off = 0;
@@ -214,6 +217,7 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
   L.dw_part = off; off += round256(P * cdiv(I, kBN) * 4);
+  L.maps = off; off += round256(static_cast<size_t>(4) * E * sizeof(CUtensorMap));
   L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
   L.total = off;
   return L;
@@ -480,10 +484,15 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     ProfScope ps(kProfCombineDx, stream);
     if (launch_combine(dXp, pair_pos, T, k, H, dX, stream, dev->num_sms) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  // 6. weight gradients, K = the expert's rows
+  // 6. weight gradients, K = the expert's rows. Each launch first writes
+  //    per-expert copies of its two tensor maps, clipped at the segment end.
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(w8 + L.maps);
   {
     GemmParams wg = base_params(E, P, offsets);
     if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64) || !make_map(&wg.tmB, Xp, H, P, 64, 64)) return MOE_ERR_CUDA;
+    build_expert_maps_kernel<<<cdiv(2 * E, 8), 256, 0, stream>>>(wg.tmA, wg.tmB, offsets, E, maps);
+    if (launch_status()) return MOE_ERR_CUDA;
+    wg.expert_maps = maps;
     wg.M = 2 * I;
     wg.N = H;
     wg.I = I;
@@ -492,13 +501,15 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     wg.out = dW_gu;
     wg.out_ld = H;
     wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
-    const int tiles = E * wg.m_tiles * wg.n_tiles;
-    if (int st = launch_gemm<kBwdWgrad>(wg, tiles < dev->num_sms ? tiles : dev->num_sms, stream, kProfWgradGateUp))
-      return st;
+    const int64_t tiles = static_cast<int64_t>(E) * wg.m_tiles * wg.n_tiles;
+    if (int st = launch_gemm<kBwdWgrad>(wg, pair_grid(tiles, dev->num_sms), stream, kProfWgradGateUp)) return st;
   }
   {
     GemmParams wd = base_params(E, P, offsets);
     if (!make_map(&wd.tmA, dYp, H, P, 64, 64) || !make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
+    build_expert_maps_kernel<<<cdiv(2 * E, 8), 256, 0, stream>>>(wd.tmA, wd.tmB, offsets, E, maps + 2 * E);
+    if (launch_status()) return MOE_ERR_CUDA;
+    wd.expert_maps = maps + 2 * E;
     wd.M = H;
     wd.N = I;
     wd.I = I;
@@ -507,9 +518,8 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     wd.out = dW_d;
     wd.out_ld = I;
     wd.out_expert_stride = static_cast<int64_t>(H) * I;
-    const int tiles = E * wd.m_tiles * wd.n_tiles;
-    if (int st = launch_gemm<kBwdWgrad>(wd, tiles < dev->num_sms ? tiles : dev->num_sms, stream, kProfWgradDown))
-      return st;
+    const int64_t tiles = static_cast<int64_t>(E) * wd.m_tiles * wd.n_tiles;
+    if (int st = launch_gemm<kBwdWgrad>(wd, pair_grid(tiles, dev->num_sms), stream, kProfWgradDown)) return st;
   }
   // 7. router logits gradient
   {

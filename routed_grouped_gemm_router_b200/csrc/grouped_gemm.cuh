@@ -11,8 +11,9 @@
 //    even CTA issues the MMA for both, and each CTA's TMEM receives its 128
 //    accumulator rows. Per CTA a 64-deep K step is 32 KiB, so a 6-deep
 //    TMA ring fits in shared memory;
-//  * 6 warps per CTA: warp 0 issues TMA loads, warp 1 issues MMAs (even CTA)
-//    and owns the TMEM allocation, warps 2-5 run the epilogue;
+//  * 10 warps per CTA: warp 0 issues TMA loads (and L2 prefetches ahead of
+//    them), warp 1 issues MMAs (even CTA) and owns the TMEM allocation,
+//    warps 2-9 run the epilogue, two per TMEM sub-partition;
 //  * both CTAs' loads complete on the even CTA's "full" mbarrier; the MMA
 //    warp's commits release the "empty" barriers of both CTAs; the fp32
 //    accumulator is double-buffered in TMEM (2 x 256 columns) so the
@@ -52,15 +53,18 @@ constexpr int kStages = 6;
 constexpr int kATileBytes = kBMc * kBK * 2;  // 16 KiB
 constexpr int kBTileBytes = kBNc * kBK * 2;  // 16 KiB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;     // two per TMEM sub-partition, each half of the columns
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kPrefetchAhead = 8;  // K blocks the L2 prefetch runs ahead of the loads
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
 constexpr int kNumBarriers = 2 * kStages + 5;
-// Epilogue staging: per epilogue warp 32 rows x 32 fp32 with a 36-float row
+// Epilogue staging: per epilogue warp 32 rows x 32 bf16 at an 80-byte row
 // stride, so both the row-wise 16-byte writes (8 lanes = 8 rows per phase)
 // and the transposed 16-byte reads (8 lanes = 8 rows per phase) hit 8
 // distinct bank groups.
-constexpr int kStageStride = 36;
+constexpr int kStageStrideBytes = 80;
+constexpr int kStageWarpBytes = 32 * kStageStrideBytes;
 
 struct GemmParams {
   CUtensorMap tmA;
@@ -84,12 +88,12 @@ struct GemmParams {
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
   const uint16_t* h_in;       // BwdDgradDown: h
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
-  float* dw_part;             // BwdDgradDown: [P, n_tiles] partial routing-weight grads
+  float* dw_part;             // BwdDgradDown: [P, 2 * n_tiles] partial routing-weight grads
 };
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
   return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes + kNumBarriers * 8 + 16 +
-         2 * static_cast<size_t>(E + 1) * 4 + 16 + 4 * 32 * kStageStride * 4;
+         2 * static_cast<size_t>(E + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * kStageWarpBytes;
 }
 
 struct TileInfo {
@@ -151,32 +155,28 @@ __device__ __forceinline__ void unpack8(const uint4 i, float* v) {
   v[6] = bf16lo(i.w); v[7] = bf16hi(i.w);
 }
 
-__device__ __forceinline__ void stage_row(float* stg, int lane, const uint32_t (&v)[32]) {
-  float* rp = stg + lane * kStageStride;
+// Row domain -> staging: the thread's 32 values of its row, rounded to bf16.
+__device__ __forceinline__ void stage_row(uint8_t* stg, int lane, const float (&v)[32]) {
+  uint8_t* rp = stg + lane * kStageStrideBytes;
 #pragma unroll
-  for (int m = 0; m < 8; ++m)
-    *reinterpret_cast<uint4*>(rp + 4 * m) = make_uint4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+  for (int m = 0; m < 4; ++m) {
+    uint4 o;
+    o.x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
+    o.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
+    o.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
+    o.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
+    *reinterpret_cast<uint4*>(rp + 16 * m) = o;
+  }
 }
 
-__device__ __forceinline__ void stage_row(float* stg, int lane, const float (&v)[32]) {
-  float* rp = stg + lane * kStageStride;
-#pragma unroll
-  for (int m = 0; m < 8; ++m)
-    *reinterpret_cast<float4*>(rp + 4 * m) = make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
-}
-
-// 8 consecutive staged values of row r starting at column 8*q.
-__device__ __forceinline__ void read_transposed(const float* stg, int r, int q, float (&o)[8]) {
-  const float* rp = stg + r * kStageStride + q * 8;
-  const float4 a = *reinterpret_cast<const float4*>(rp);
-  const float4 b = *reinterpret_cast<const float4*>(rp + 4);
-  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
-  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+// Transposed domain: 8 bf16 of staged row r starting at column 8*q.
+__device__ __forceinline__ uint4 read_piece(const uint8_t* stg, int r, int q) {
+  return *reinterpret_cast<const uint4*>(stg + r * kStageStrideBytes + q * 16);
 }
 
 // Stores one 32-column chunk (row domain values v, thread = row) as bf16 to
 // base[(row0 + r) * ld + col0 + c] for the warp's valid rows and c < ncols.
-__device__ __forceinline__ void emit_chunk(float* stg, const float (&v)[32], uint16_t* base, int64_t row0,
+__device__ __forceinline__ void emit_chunk(uint8_t* stg, const float (&v)[32], uint16_t* base, int64_t row0,
                                            int64_t ld, int col0, int ncols, int wrows, int tr_row, int tr_q,
                                            int lane) {
   stage_row(stg, lane, v);
@@ -185,11 +185,7 @@ __device__ __forceinline__ void emit_chunk(float* stg, const float (&v)[32], uin
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = i * 8 + tr_row;
-    if (r < wrows && col < ncols) {
-      float o[8];
-      read_transposed(stg, r, tr_q, o);
-      store8_bf16(base + (row0 + r) * ld + col, o);
-    }
+    if (r < wrows && col < ncols) *reinterpret_cast<uint4*>(base + (row0 + r) * ld + col) = read_piece(stg, r, tr_q);
   }
   __syncwarp();
 }
@@ -242,7 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
   int* s_tstart = s_off + (p.E + 1);
-  float* s_stage = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 15) & ~uintptr_t(15));
+  uint8_t* s_stage = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -258,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 2 * 128);
+      mbar_init(&tempty_bar[a], 2 * 32 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -303,54 +299,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
+    // Loads K block kb of tile ti (this CTA's A half and B half) into a ring
+    // stage, or with prefetch_only just asks TMA to bring the same boxes into
+    // L2. A prefetch cursor runs kPrefetchAhead K blocks (across tile
+    // boundaries) ahead of the loads so first touches of weight and
+    // activation tiles start their DRAM reads early.
+    auto issue = [&](const TileInfo& ti, int kb, bool prefetch_only, uint8_t* a_dst, uint8_t* b_dst, uint32_t fb) {
+      const CUtensorMap* mapA = &p.tmA;
+      const CUtensorMap* mapB = &p.tmB;
+      if constexpr (kWgrad) {
+        mapA = p.expert_maps + ti.e;
+        mapB = p.expert_maps + p.E + ti.e;
+      }
+      const int kx = kb * kBK;
+      int ax, ay, bx, by, nbox_a = 1, nbox_b = 1;
+      if constexpr (KIND == kFwdGateUp) {
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
+        // even CTA: the tile's 128 gate rows; odd CTA: the matching up rows
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * p.I;
+      } else if constexpr (KIND == kFwdDown) {
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
+      } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
+        bx = ti.n_blk * kBN + static_cast<int>(rank) * kBNc; by = ti.e * p.b_rows + kx;
+        nbox_b = 2;
+      } else {  // wgrad: K rows are the expert's permuted rows
+        ax = ti.m_blk * kBM + static_cast<int>(rank) * kBMc; ay = ti.row0 + kx;
+        bx = ti.n_blk * kBN + static_cast<int>(rank) * kBNc; by = ay;
+        nbox_a = 2;
+        nbox_b = 2;
+      }
+      for (int c = 0; c < nbox_a; ++c) {
+        if (prefetch_only) tma_prefetch_2d(mapA, ax + 64 * c, ay);
+        else tma_load_2d_pair(a_dst + 8192 * c, mapA, fb, ax + 64 * c, ay);
+      }
+      for (int c = 0; c < nbox_b; ++c) {
+        if (prefetch_only) tma_prefetch_2d(mapB, bx + 64 * c, by);
+        else tma_load_2d_pair(b_dst + 8192 * c, mapB, fb, bx + 64 * c, by);
+      }
+    };
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
+      // prefetch cursor: tile pf_t, K block pf_kb; pf_lead = blocks ahead of the loads
+      int pf_t = pair, pf_kb = 0, pf_lead = 0;
+      TileInfo pf_ti;
+      if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
       for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
         const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
-        const CUtensorMap* mapA = &p.tmA;
-        const CUtensorMap* mapB = &p.tmB;
         if constexpr (kWgrad) {
           if (ti.num_kb == 0) continue;
-          mapA = p.expert_maps + ti.e;
-          mapB = p.expert_maps + p.E + ti.e;
-          tensormap_acquire(mapA);
-          tensormap_acquire(mapB);
+          tensormap_acquire(p.expert_maps + ti.e);
+          tensormap_acquire(p.expert_maps + p.E + ti.e);
         }
         for (int kb = 0; kb < ti.num_kb; ++kb) {
+          while (pf_lead < kPrefetchAhead && pf_t < total_tiles) {
+            if (pf_kb < pf_ti.num_kb) {
+              if constexpr (kWgrad) {
+                if (pf_kb == 0) {
+                  tensormap_acquire(p.expert_maps + pf_ti.e);
+                  tensormap_acquire(p.expert_maps + p.E + pf_ti.e);
+                }
+              }
+              issue(pf_ti, pf_kb, true, nullptr, nullptr, 0);
+              ++pf_kb;
+              ++pf_lead;
+            } else {
+              pf_t += num_pairs;
+              pf_kb = 0;
+              if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
+            }
+          }
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             report(MOE_ERR_TIMEOUT);
             *s_abort = 1;
             break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
-          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-          uint8_t* a_dst = sA + stage * kATileBytes;
-          uint8_t* b_dst = sB + stage * kBTileBytes;
-          const int kx = kb * kBK;
-          if constexpr (KIND == kFwdGateUp) {
-            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
-            // even CTA: the tile's 128 gate rows; odd CTA: the matching up rows
-            tma_load_2d_pair(b_dst, mapB, fb, kx, ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * p.I);
-          } else if constexpr (KIND == kFwdDown) {
-            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
-            tma_load_2d_pair(b_dst, mapB, fb, kx, ti.e * p.b_rows + ti.n_blk * kBN + static_cast<int>(rank) * kBNc);
-          } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
-            tma_load_2d_pair(a_dst, mapA, fb, kx, ti.row0 + static_cast<int>(rank) * kBMc);
-            const int krow = ti.e * p.b_rows + kx;
-            const int n0 = ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
-            tma_load_2d_pair(b_dst, mapB, fb, n0, krow);
-            tma_load_2d_pair(b_dst + 8192, mapB, fb, n0 + 64, krow);
-          } else {  // wgrad: K rows are the expert's permuted rows
-            const int krow = ti.row0 + kx;
-            const int m0 = ti.m_blk * kBM + static_cast<int>(rank) * kBMc;
-            const int n0 = ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
-            tma_load_2d_pair(a_dst, mapA, fb, m0, krow);
-            tma_load_2d_pair(a_dst + 8192, mapA, fb, m0 + 64, krow);
-            tma_load_2d_pair(b_dst, mapB, fb, n0, krow);
-            tma_load_2d_pair(b_dst + 8192, mapB, fb, n0 + 64, krow);
-          }
+          issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes,
+                mapa_shared(smem_u32(&full_bar[stage]), 0));
+          if (pf_lead > 0) --pf_lead;
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -436,16 +466,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------- epilogue
     // Thread (warp w, lane l) reads TMEM lane 32*(w%4)+l: one accumulator row
-    // ("row domain"). Every 32-column chunk is staged through the warp's own
+    // ("row domain"); the two warps of a sub-partition split the columns.
+    // Every 32-column chunk is rounded to bf16, staged through the warp's own
     // shared buffer and read back transposed ("transposed domain"): lane l
     // then owns rows 8*i + (l%8), i = 0..3, and columns 8*(l/8)..+7 of the
     // chunk, so each global load/store instruction covers 8 rows x 64
     // contiguous bytes instead of 32 rows x 16 bytes.
     const int sub = warp & 3;
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
     const int tr_row = lane & 7;
     const int tr_q = lane >> 3;
-    float* stg = s_stage + (warp - 2) * 32 * kStageStride;
+    uint8_t* stg = s_stage + (warp - 2) * kStageWarpBytes;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / 2;  // chunks per warp
     int tcount = 0;
     for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
@@ -457,10 +490,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + cta_row0
                                    : static_cast<int64_t>(ti.row0) + cta_row0;
       uint16_t* out_base = kWgrad ? p.out + ti.e * p.out_expert_stride : p.out;
+      const int ch0 = half * kChunks;  // first 32-column chunk of this warp
       if constexpr (kWgrad) {
         if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero
-          for (int c = 0; c < kBN; c += 32) {
-            const int col = ti.n_blk * kBN + c + tr_q * 8;
+          for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
+            const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = i * 8 + tr_row;
@@ -483,7 +517,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // their latency hides behind the main loop
       uint4 dd_cur[12];
       if constexpr (KIND == kBwdDgradDown)
-        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + tr_q * 8, tr_row, dd_cur);
+        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + ch0 * 32 + tr_q * 8, tr_row, dd_cur);
 
       const int acc = tcount & 1;
       if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
@@ -493,10 +527,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(sub * 32) << 16);
+
       if constexpr (KIND == kFwdGateUp) {
         const int I = p.I;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
           uint32_t g[32], u[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, g);
           tmem_ld_32x32b_x32(taddr + 128 + ch * 32, u);
@@ -525,21 +560,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) wrow[i] = __shfl_sync(0xffffffffu, wq, i * 8 + tr_row);
 #pragma unroll 1
-        for (int ch = 0; ch < kBN / 32; ++ch) {
+        for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
           const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
           uint4 nxt[12];
-          if (ch + 1 < kBN / 32) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
+          if (ch + 1 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
           uint32_t a[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
-          stage_row(stg, lane, a);
+          float av[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) av[j] = __uint_as_float(a[j]);
+          stage_row(stg, lane, av);
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int r = i * 8 + tr_row;
             if (r < wrows && col < I) {
               float dhp[8], gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
-              read_transposed(stg, r, tr_q, dhp);
+              unpack8(read_piece(stg, r, tr_q), dhp);
               unpack8(dd_cur[3 * i], gv);
               unpack8(dd_cur[3 * i + 1], uv);
               unpack8(dd_cur[3 * i + 2], hv);
@@ -562,26 +600,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
         }
-        // each row's partial dot product is spread over the 4 lanes with the same l%8
+        // each row's partial dot product is spread over the 4 lanes with the
+        // same l%8; the two column halves write separate slots
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 8);
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 16);
           const int r = i * 8 + tr_row;
-          if (tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * p.n_tiles + ti.n_blk] = dwp[i];
+          if (tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
         }
       } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
 #pragma unroll 1
-        for (int ch = 0; ch < kBN / 32; ++ch) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(taddr + ch * 32, a);
+        for (int ch = ch0; ch < ch0 + kChunks; ch += 2) {
+          uint32_t a0[32], a1[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, a0);
+          tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, a1);
           tmem_ld_wait();
           const int col0 = ti.n_blk * kBN + ch * 32;
-          if (col0 >= p.N) continue;  // warp-uniform
           float v[32];
+          if (col0 < p.N) {  // warp-uniform
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a[j]);
-          emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane);
+            for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a0[j]);
+            emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane);
+          }
+          if (col0 + 32 < p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a1[j]);
+            emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0 + 32, p.N, wrows, tr_row, tr_q, lane);
+          }
         }
       }
       tc_fence_before();

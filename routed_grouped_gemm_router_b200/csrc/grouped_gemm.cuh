@@ -53,9 +53,19 @@ constexpr int kStages = 6;
 constexpr int kATileBytes = kBMc * kBK * 2;  // 16 KiB
 constexpr int kBTileBytes = kBNc * kBK * 2;  // 16 KiB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kEpiWarps = 8;     // two per TMEM sub-partition, each half of the columns
+// Epilogue warps: 4 (one per TMEM sub-partition) or 8 (two per sub-partition,
+// each half of the columns).
+#ifndef MOE_EPI_WARPS
+#define MOE_EPI_WARPS 8
+#endif
+// K blocks the L2 prefetch cursor runs ahead of the TMA loads (0: off).
+#ifndef MOE_PREFETCH_AHEAD
+#define MOE_PREFETCH_AHEAD 0
+#endif
+constexpr int kEpiWarps = MOE_EPI_WARPS;
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "4 or 8 epilogue warps");
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
-constexpr int kPrefetchAhead = 8;  // K blocks the L2 prefetch runs ahead of the loads
+constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
 constexpr int kNumBarriers = 2 * kStages + 5;
@@ -209,8 +219,11 @@ __device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t wro
   }
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// silu(x) = x / (1 + e^-x) and the logistic sigmoid, with CUDA's fast exp and
+// division intrinsics (a few ulp; for x << 0 the denominator overflows to
+// inf and both return 0).
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
@@ -473,12 +486,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // chunk, so each global load/store instruction covers 8 rows x 64
     // contiguous bytes instead of 32 rows x 16 bytes.
     const int sub = warp & 3;
-    const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    const int half = kEpiWarps == 8 ? (warp - 2) >> 2 : 0;  // which half of the tile's columns
     const int tr_row = lane & 7;
     const int tr_q = lane >> 3;
     uint8_t* stg = s_stage + (warp - 2) * kStageWarpBytes;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
-    constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / 2;  // chunks per warp
+    constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / (kEpiWarps / 4);  // chunks per warp
     int tcount = 0;
     for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
@@ -607,7 +620,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 8);
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 16);
           const int r = i * 8 + tr_row;
-          if (tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
+          if (tr_q == 0 && r < wrows)
+            p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
+          if (kEpiWarps == 4 && tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + 1] = 0.f;
         }
       } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
 #pragma unroll 1

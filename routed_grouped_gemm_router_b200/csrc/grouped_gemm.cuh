@@ -69,11 +69,11 @@ constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
 constexpr int kNumBarriers = 2 * kStages + 5;
-// Epilogue staging: per epilogue warp 32 rows x 32 bf16 at an 80-byte row
-// stride, so both the row-wise 16-byte writes (8 lanes = 8 rows per phase)
-// and the transposed 16-byte reads (8 lanes = 8 rows per phase) hit 8
-// distinct bank groups.
-constexpr int kStageStrideBytes = 80;
+// Epilogue staging: per epilogue warp 32 rows x 32 bf16 (64 bytes per row).
+// The four 16-byte pieces of row r are stored at piece (m ^ ((r >> 1) & 3)),
+// which keeps both the row-wise writes (8 rows per quarter-warp phase) and
+// the transposed reads (2 rows x 4 pieces per phase) free of bank conflicts.
+constexpr int kStageStrideBytes = 64;
 constexpr int kStageWarpBytes = 32 * kStageStrideBytes;
 
 struct GemmParams {
@@ -168,6 +168,7 @@ __device__ __forceinline__ void unpack8(const uint4 i, float* v) {
 // Row domain -> staging: the thread's 32 values of its row, rounded to bf16.
 __device__ __forceinline__ void stage_row(uint8_t* stg, int lane, const float (&v)[32]) {
   uint8_t* rp = stg + lane * kStageStrideBytes;
+  const int sw = (lane >> 1) & 3;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     uint4 o;
@@ -175,17 +176,19 @@ __device__ __forceinline__ void stage_row(uint8_t* stg, int lane, const float (&
     o.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
     o.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
     o.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
-    *reinterpret_cast<uint4*>(rp + 16 * m) = o;
+    *reinterpret_cast<uint4*>(rp + 16 * (m ^ sw)) = o;
   }
 }
 
 // Transposed domain: 8 bf16 of staged row r starting at column 8*q.
 __device__ __forceinline__ uint4 read_piece(const uint8_t* stg, int r, int q) {
-  return *reinterpret_cast<const uint4*>(stg + r * kStageStrideBytes + q * 16);
+  return *reinterpret_cast<const uint4*>(stg + r * kStageStrideBytes + 16 * (q ^ ((r >> 1) & 3)));
 }
 
 // Stores one 32-column chunk (row domain values v, thread = row) as bf16 to
 // base[(row0 + r) * ld + col0 + c] for the warp's valid rows and c < ncols.
+// In the transposed domain lane l writes row 8*i + l/4, columns 8*(l%4)..+7:
+// every quarter-warp writes two rows of 64 contiguous bytes.
 __device__ __forceinline__ void emit_chunk(uint8_t* stg, const float (&v)[32], uint16_t* base, int64_t row0,
                                            int64_t ld, int col0, int ncols, int wrows, int tr_row, int tr_q,
                                            int lane) {
@@ -267,7 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 2 * 32 * kEpiWarps);
+      mbar_init(&tempty_bar[a], 2 * kEpiWarps);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -482,13 +485,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ("row domain"); the two warps of a sub-partition split the columns.
     // Every 32-column chunk is rounded to bf16, staged through the warp's own
     // shared buffer and read back transposed ("transposed domain"): lane l
-    // then owns rows 8*i + (l%8), i = 0..3, and columns 8*(l/8)..+7 of the
-    // chunk, so each global load/store instruction covers 8 rows x 64
-    // contiguous bytes instead of 32 rows x 16 bytes.
+    // then owns rows 8*i + l/4, i = 0..3, and columns 8*(l%4)..+7 of the
+    // chunk, so each quarter-warp of a 16-byte global access covers two rows
+    // of 64 contiguous bytes.
     const int sub = warp & 3;
     const int half = kEpiWarps == 8 ? (warp - 2) >> 2 : 0;  // which half of the tile's columns
-    const int tr_row = lane & 7;
-    const int tr_q = lane >> 3;
+    const int tr_row = lane >> 2;  // transposed domain: row 8*i + tr_row
+    const int tr_q = lane & 3;     // transposed domain: columns 8*tr_q..+7 of the chunk
     uint8_t* stg = s_stage + (warp - 2) * kStageWarpBytes;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / (kEpiWarps / 4);  // chunks per warp
@@ -614,11 +617,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
         }
         // each row's partial dot product is spread over the 4 lanes with the
-        // same l%8; the two column halves write separate slots
+        // same l/4; the two column halves write separate slots
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 8);
-          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 16);
+          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 1);
+          dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 2);
           const int r = i * 8 + tr_row;
           if (tr_q == 0 && r < wrows)
             p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
@@ -646,7 +649,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive_cluster(leader_tempty0 + acc * 8);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);
       ++tcount;
     }
   }

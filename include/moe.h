@@ -115,6 +115,29 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
                 size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_permute_noalloc -- moe_permute without a workspace argument, for
+ * callers that cannot allocate device memory: a host program or plug-in that
+ * links only this library and has no device allocator of its own, or code
+ * that must not call cudaMalloc (it synchronises the device). The pages have
+ * no counterpart; this is a calling convenience of this library.
+ *
+ * Arguments and results are exactly those of moe_permute (same kernels).
+ * The scratch comes from one fixed 1 MiB device array inside the library
+ * (held on every GPU that loads the library until the process exits), so the
+ * problem must satisfy ceil(T*k / 2048) * E <= 262144 (for E = 128: up to
+ * 4,194,304 pairs); larger problems return MOE_ERR_WORKSPACE and launch
+ * nothing. The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture. All calls share the array: calls whose executions
+ * overlap on the GPU (other streams or host threads on the same device) race
+ * on it. Leftover contents from earlier calls are harmless: every value read
+ * is written earlier in the same call.
+ */
+int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                        int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X, int H, moe_bf16* Xp,
+                        moe_stream_t stream);
+
+/*
  * moe_experts_fwd -- the two persistent grouped GEMMs over the expert
  * segments (tcgen05 tensor cores, TMEM accumulators, TMA-fed tiles; experts
  * with no rows cost nothing).

@@ -28,6 +28,8 @@ _SIGNATURES = {
     "moe_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_permute": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void, _c_void,
                              _c_int, _c_void, _c_void, _c_size, _c_void]),
+    "moe_permute_noalloc": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void,
+                                     _c_void, _c_int, _c_void, _c_void]),
     "moe_experts_fwd": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
                                  _c_void, _c_void, _c_void, _c_void, _c_void, _c_void]),
     "moe_combine": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void]),

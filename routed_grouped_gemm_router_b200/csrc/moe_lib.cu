@@ -319,6 +319,57 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: moe_permute for callers that cannot allocate device
+// memory. Some callers have no way to obtain device scratch: a host program
+// or plug-in that links only this C library and holds no device allocator,
+// or code running where a device allocation would stall or is not allowed
+// (cudaMalloc synchronises the device). This entry point takes its scratch
+// from a fixed, file-scope device array instead of the caller's workspace.
+//
+// The array is a module global: every GPU that loads this library holds its
+// 1 MiB until the process exits. All calls share it, so calls whose
+// executions overlap on the GPU (different streams, or different host threads
+// on one device) race on it; one stream at a time is safe because the
+// kernels of one call finish before the next call's kernels start. The
+// histogram pass overwrites every element it later reads, so the contents
+// left by the previous call never need clearing.
+constexpr int kNoAllocPermuteScratchInts = 262144;  // 1 MiB
+static __device__ __align__(256) int g_permute_scratch[kNoAllocPermuteScratchInts];
+
+namespace {
+// Device address of g_permute_scratch for each device, looked up on the first
+// call made with that device current (host code may not use the symbol's name
+// as a device pointer).
+int* g_permute_scratch_ptr[kMaxDevices] = {};
+std::mutex g_permute_scratch_mu;
+
+int permute_scratch_device_ptr(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_permute_scratch_mu);
+  if (g_permute_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_permute_scratch_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_permute_scratch_ptr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                        int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X, int H, moe_bf16* Xp,
+                        moe_stream_t stream) {
+  if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_permute_workspace_bytes(T, E, k);
+  if (need > sizeof(int) * static_cast<size_t>(kNoAllocPermuteScratchInts)) return MOE_ERR_WORKSPACE;
+  int* scratch = nullptr;
+  if (int st = permute_scratch_device_ptr(&scratch)) return st;
+  return moe_permute(topk_idx, T, E, k, counts, offsets, sorted_pair, pair_pos, X, H, Xp, scratch,
+                     sizeof(int) * static_cast<size_t>(kNoAllocPermuteScratchInts), stream);
+}
+
 int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
                     int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
                     moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {

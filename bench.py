@@ -189,6 +189,25 @@ def step_flops(wl):
     return wl.flops_fwd() + (wl.flops_bwd() if wl.backward else 0.0)
 
 
+def world_info():
+    """(world size, rank, local rank) from the torch.distributed.run environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank values (device-timed milliseconds)."""
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tflops(world, flops_per_step, steps, total_ms):
+    """Whole-job throughput: every rank processed `steps` steps of its own batch."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def run_reference(args, wl, rank):
     """The oracle timed on the host cores (rank 0 only)."""
     if rank != 0:
@@ -248,9 +267,7 @@ def main():
         wl = type(wl)(name, T, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts,
                       wl.backward and not args.forward_only)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = world_info()
     if args.impl == "reference":
         run_reference(args, wl, rank)
         return
@@ -390,9 +407,8 @@ def main():
     clocks = sampler.stop() if sampler else None
 
     if world > 1:
-        t = torch.tensor([total_ms, e2e_ms or 0.0], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = t[0].item(), (t[1].item() if e2e_ms is not None else None)
+        t_max, e_max = max_over_ranks([total_ms, e2e_ms or 0.0], dev)
+        total_ms, e2e_ms = t_max, (e_max if e2e_ms is not None else None)
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -400,8 +416,8 @@ def main():
 
     flops = step_flops(wl)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = world * flops * args.steps / (e2e_ms * 1e-3) / 1e12 if e2e_ms else None
+    value = aggregate_tflops(world, flops, args.steps, total_ms)
+    e2e_value = aggregate_tflops(world, flops, args.steps, e2e_ms) if e2e_ms else None
     peaks, peaks_src = read_peaks()
 
     # dominant kernel: most device time over the timed region

@@ -200,6 +200,16 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_selftest_wait_timeout -- diagnostics: enqueues one kernel that waits on
+ * a barrier nothing signals, using the same bounded wait as the pipeline
+ * kernels but with a limit of limit_ms (1..2000) milliseconds. When the limit
+ * passes the kernel records MOE_ERR_TIMEOUT in the device status word and
+ * exits, so moe_last_device_status(stream) then returns MOE_ERR_TIMEOUT and
+ * the context stays usable. No counterpart on the pages.
+ */
+int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream);
+
+/*
  * Per-kernel timing with CUDA events recorded on the launching stream around
  * every kernel launch (off by default; measurement only, no effect on results).
  * moe_profile_enable(1) starts recording and clears earlier records.

@@ -35,6 +35,7 @@ _SIGNATURES = {
     "moe_combine": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void]),
     "moe_layer_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
+    "moe_selftest_wait_timeout": (_c_int, [_c_int, _c_void]),
     "moe_profile_enable": (_c_int, [_c_int]),
     "moe_profile_read": (_c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
     "moe_profile_kernel_name": (ctypes.c_char_p, [_c_int]),

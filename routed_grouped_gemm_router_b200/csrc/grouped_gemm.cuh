@@ -66,6 +66,17 @@ constexpr int kEpiWarps = MOE_EPI_WARPS;
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "4 or 8 epilogue warps");
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
+// Epilogue outputs are written with the streaming hint (evict-first in L2)
+// so they do not push reused operand tiles out of L2.
+#ifndef MOE_STREAM_STORES
+#define MOE_STREAM_STORES 1
+#endif
+// Raster of the row-grouped tiles inside an expert: 0 = N block fastest
+// (concurrent pairs share A rows), 1 = row block fastest (concurrent pairs
+// share a weight tile).
+#ifndef MOE_TILE_M_FASTEST
+#define MOE_TILE_M_FASTEST 0
+#endif
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
 constexpr int kNumBarriers = 2 * kStages + 5;
@@ -134,8 +145,14 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     }
     ti.e = lo;
     const int local = t - s_tstart[lo];
+#if MOE_TILE_M_FASTEST
+    const int m_tiles_e = (s_off[lo + 1] - s_off[lo] + kBM - 1) / kBM;
+    ti.n_blk = local / m_tiles_e;
+    ti.m_blk = local - ti.n_blk * m_tiles_e;
+#else
     ti.m_blk = local / p.n_tiles;
     ti.n_blk = local - ti.m_blk * p.n_tiles;
+#endif
     ti.row0 = s_off[lo] + ti.m_blk * kBM;
     ti.rows = s_off[lo + 1] - ti.row0;
     ti.num_kb = (p.K + kBK - 1) / kBK;
@@ -149,13 +166,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
+__device__ __forceinline__ void store16(uint16_t* dst, uint4 v) {
+#if MOE_STREAM_STORES
+  __stcs(reinterpret_cast<uint4*>(dst), v);
+#else
+  *reinterpret_cast<uint4*>(dst) = v;
+#endif
+}
+
 __device__ __forceinline__ void store8_bf16(uint16_t* dst, const float* v) {
   uint4 o;
   o.x = pack_bf16(v[0], v[1]);
   o.y = pack_bf16(v[2], v[3]);
   o.z = pack_bf16(v[4], v[5]);
   o.w = pack_bf16(v[6], v[7]);
-  *reinterpret_cast<uint4*>(dst) = o;
+  store16(dst, o);
 }
 
 __device__ __forceinline__ void unpack8(const uint4 i, float* v) {
@@ -198,7 +223,7 @@ __device__ __forceinline__ void emit_chunk(uint8_t* stg, const float (&v)[32], u
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = i * 8 + tr_row;
-    if (r < wrows && col < ncols) *reinterpret_cast<uint4*>(base + (row0 + r) * ld + col) = read_piece(stg, r, tr_q);
+    if (r < wrows && col < ncols) store16(base + (row0 + r) * ld + col, read_piece(stg, r, tr_q));
   }
   __syncwarp();
 }

@@ -23,6 +23,25 @@
 #include "router_bwd.cuh"
 
 namespace moe {
+
+// Waits on an mbarrier that nothing ever arrives at, with the library's
+// bounded wait shortened to `limit_ns`; when the limit passes it records
+// MOE_ERR_TIMEOUT in the device status word and returns. Exercises the
+// failure path of every pipeline wait without hanging the device.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbarrier_init();
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(&bar, 0)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      report(MOE_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
 namespace {
 
 // ------------------------------------------------------------------ helpers
@@ -582,6 +601,14 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     if (launch_status()) return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  return launch_status();
 }
 
 int moe_profile_enable(int on) {

@@ -71,15 +71,14 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
           be = e;
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-          bv = ov;
-          be = oe;
-        }
-      }
+      // Warp argmax in two reductions: the largest logit (as an order-
+      // preserving integer key; -0.0 is folded into +0.0 so signed zeros tie),
+      // then the smallest expert index among the lanes holding it.
+      const float cv = (bv == 0.0f) ? 0.0f : bv;
+      const uint32_t bits = __float_as_uint(cv);
+      const uint32_t key = (be == 0x7fffffff) ? 0u : ((bits & 0x80000000u) ? ~bits : (bits | 0x80000000u));
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+      be = static_cast<int>(__reduce_min_sync(0xffffffffu, key == kmax ? static_cast<uint32_t>(be) : 0xffffffffu));
       // owner lane marks the winner taken; every lane learns its probability
       float pwin = 0.f;
       if ((be & 31) == lane) {

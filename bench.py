@@ -57,7 +57,7 @@ def kernel_work(name, wl):
         "gather_x": T * H * 2 + P * H * 2 + P * 4, "gather_dy": T * H * 2 + P * H * 2 + P * 4,
         "combine_y": P * H * 2 + T * H * 2 + P * 4, "combine_dx": P * H * 2 + T * H * 2 + P * 4,
         "route": T * E * 4 * 2 + T * k * 8,
-        "router_bwd": T * E * 4 * 2 + T * k * 12 + P * 16 * ((I + 255) // 256),
+        "router_bwd": T * E * 4 * 2 + T * k * 12 + P * 8 * ((I + 255) // 256),
         "permute_count": P * 4, "permute_scan": E * 8, "permute_scatter": P * 12,
     }
     return "hbm", float(nbytes.get(name, 0))

@@ -109,7 +109,7 @@ struct GemmParams {
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
   const uint16_t* h_in;       // BwdDgradDown: h
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
-  float* dw_part;             // BwdDgradDown: [P, 4 * n_tiles] partial routing-weight grads
+  float* dw_part;             // BwdDgradDown: [P, 2 * n_tiles] partial routing-weight grads
 };
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
@@ -122,7 +122,6 @@ struct TileInfo {
   int row0;     // first permuted row of the pair tile (row-grouped) / first K row (wgrad)
   int rows;     // rows of the segment from row0 on (row-grouped) / rows of the segment (wgrad)
   int num_kb;   // K blocks
-  bool half;    // row-grouped tile with <= 128 rows: pair MMA with M = 128 (64 rows per CTA)
 };
 
 template <int KIND>
@@ -138,7 +137,6 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.row0 = s_off[ti.e];
     ti.rows = s_off[ti.e + 1] - ti.row0;
     ti.num_kb = (ti.rows + kBK - 1) / kBK;
-    ti.half = false;
   } else {
     int lo = 0, hi = p.E;  // s_tstart[lo] <= t < s_tstart[hi]
     while (hi - lo > 1) {
@@ -158,7 +156,6 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.row0 = s_off[lo] + ti.m_blk * kBM;
     ti.rows = s_off[lo + 1] - ti.row0;
     ti.num_kb = (p.K + kBK - 1) / kBK;
-    ti.half = ti.rows <= kBMc;
   }
   return ti;
 }
@@ -266,7 +263,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   constexpr bool kAMN = kWgrad;
   constexpr bool kBMN = (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || kWgrad);
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, kAMN, kBMN);
-  constexpr uint32_t kIdescHalf = idesc_bf16_f32(kBM / 2, kBN, kAMN, kBMN);
   constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
   constexpr uint32_t kBLbo = kBMN ? 8192u : 16u;
   constexpr uint32_t kAStep = kAMN ? 2048u : 32u;  // bytes per UMMA_K step
@@ -361,26 +357,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       const int kx = kb * kBK;
       int ax, ay, bx, by, nbox_a = 1, nbox_b = 1;
-      // A rows of this CTA: 128 of a full tile, 64 of a half tile (the
-      // 128-row box then also brings the peer's rows, which the MMA ignores)
-      const int a_row = ti.row0 + static_cast<int>(rank) * (ti.half ? kBMc / 2 : kBMc);
       if constexpr (KIND == kFwdGateUp) {
-        // B half of CTA r: 64 gate rows then the matching 64 up rows of the
-        // tile's 128 output columns, so gate and up of a column always land
-        // in the same accumulator lane, for full and half tiles alike
-        const int g_row = ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * 64;
-        for (int c = 0; c < 2; ++c) {
-          if (prefetch_only) tma_prefetch_2d(mapB, kx, g_row + c * p.I);
-          else tma_load_2d_pair(b_dst + 8192 * c, mapB, fb, kx, g_row + c * p.I);
-        }
-        if (prefetch_only) tma_prefetch_2d(mapA, kx, a_row);
-        else tma_load_2d_pair(a_dst, mapA, fb, kx, a_row);
-        return;
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
+        // even CTA: the tile's 128 gate rows; odd CTA: the matching up rows
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * p.I;
       } else if constexpr (KIND == kFwdDown) {
-        ax = kx; ay = a_row;
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
         bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
       } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
-        ax = kx; ay = a_row;
+        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
         bx = ti.n_blk * kBN + static_cast<int>(rank) * kBNc; by = ti.e * p.b_rows + kx;
         nbox_b = 2;
       } else {  // wgrad: K rows are the expert's permuted rows
@@ -480,7 +465,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        const uint32_t idesc = ti.half ? kIdescHalf : kIdesc;
         bool ok = true;
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           if (!warp_wait(&full_bar[stage], phase)) {
@@ -495,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
               const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
               const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
-              umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              umma_bf16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit_pair(smem_u32(&empty_bar[stage]));
             umma_commit_pair(peer_empty0 + stage * 8);
@@ -525,45 +509,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------- epilogue
-    // Thread (warp w, lane l) reads TMEM lane 32*(w%4)+l ("row domain"). A
-    // full tile holds the CTA's 128 rows x 256 columns (lane = row); a half
-    // tile (pair MMA with M = 128) holds 64 rows, columns 0..127 in lanes
-    // 0..63 and columns 128..255 in lanes 64..127, both at TMEM columns
-    // 0..127. The two warps of a sub-partition split its columns. Every
-    // 32-column chunk is rounded to bf16, staged through the warp's shared
-    // buffer and read back transposed: lane l then owns rows 8*i + l/4 and
-    // columns 8*(l%4)..+7 of the chunk, so each quarter-warp of a 16-byte
-    // global access covers two rows of 64 contiguous bytes.
+    // Thread (warp w, lane l) reads TMEM lane 32*(w%4)+l: one accumulator row
+    // ("row domain"); the two warps of a sub-partition split the columns.
+    // Every 32-column chunk is rounded to bf16, staged through the warp's own
+    // shared buffer and read back transposed ("transposed domain"): lane l
+    // then owns rows 8*i + l/4, i = 0..3, and columns 8*(l%4)..+7 of the
+    // chunk, so each quarter-warp of a 16-byte global access covers two rows
+    // of 64 contiguous bytes.
     const int sub = warp & 3;
-    const int half_w = kEpiWarps == 8 ? (warp - 2) >> 2 : 0;  // which half of the sub-partition's columns
+    const int half = kEpiWarps == 8 ? (warp - 2) >> 2 : 0;  // which half of the tile's columns
     const int tr_row = lane >> 2;  // transposed domain: row 8*i + tr_row
     const int tr_q = lane & 3;     // transposed domain: columns 8*tr_q..+7 of the chunk
     uint8_t* stg = s_stage + (warp - 2) * kStageWarpBytes;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / (kEpiWarps / 4);  // chunks per warp
     int tcount = 0;
     for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
-      // Rows of this warp: full tile -> CTA rows rank*128 + 32*sub + [0,32);
-      // half tile -> rank*64 + 32*(sub&1) + [0,32). Columns: full tile -> all
-      // 256 (TMEM column = tile column); half tile -> tile columns
-      // 128*(sub>>1) + TMEM column.
-      const int cta_row0 = ti.half ? static_cast<int>(rank) * (kBMc / 2) + 32 * (sub & 1)
-                                   : static_cast<int>(rank) * kBMc + 32 * sub;
-      const int col_base = ti.half ? 128 * (sub >> 1) : 0;
+      // this CTA's 128 rows of the pair tile, this warp's 32 of them
+      const int cta_row0 = static_cast<int>(rank) * kBMc + sub * 32;
       const int tile_rows = kWgrad ? p.M - ti.m_blk * kBM : ti.rows;
       const int wrows = max(0, min(32, tile_rows - cta_row0));
       // first output row of this warp: permuted row (row-grouped) or dW row (wgrad)
       const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + cta_row0
                                    : static_cast<int64_t>(ti.row0) + cta_row0;
       uint16_t* out_base = kWgrad ? p.out + ti.e * p.out_expert_stride : p.out;
-      // TMEM columns of this warp, in 32-column chunks: [ch0, ch0 + nch)
-      constexpr int kTmemColsFull = (KIND == kFwdGateUp) ? 128 : kBN;  // columns one lane holds (gate/up: per half)
-      const int lane_cols = ti.half ? 128 : kTmemColsFull;
-      const int nch = lane_cols / 32 / (kEpiWarps / 4);
-      const int ch0 = half_w * nch;
+      const int ch0 = half * kChunks;  // first 32-column chunk of this warp
       if constexpr (kWgrad) {
         if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero
-          for (int ch = ch0; ch < ch0 + nch; ++ch) {
+          for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
             const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -587,7 +561,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // their latency hides behind the main loop
       uint4 dd_cur[12];
       if constexpr (KIND == kBwdDgradDown)
-        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + col_base + ch0 * 32 + tr_q * 8, tr_row, dd_cur);
+        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + ch0 * 32 + tr_q * 8, tr_row, dd_cur);
 
       const int acc = tcount & 1;
       if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
@@ -599,36 +573,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(sub * 32) << 16);
 
       if constexpr (KIND == kFwdGateUp) {
-        // Pair accumulator columns [128g, 128g+64) hold gate and
-        // [128g+64, 128g+128) up of output columns 64g..64g+63 of the tile.
-        // Full tile: every lane holds both groups g = 0, 1; the warp with
-        // column half h takes group g = h as two 32-column chunks. Half tile:
-        // lanes 0..63 hold group 0 and lanes 64..127 group 1, each at TMEM
-        // columns 0..127; the warp takes one chunk at offset 32*h.
         const int I = p.I;
-        const int n_gu = ti.half ? 1 : 2;
 #pragma unroll 1
-        for (int c = 0; c < n_gu; ++c) {
-          const int g = ti.half ? 0 : half_w;
-          const int off = ti.half ? 32 * half_w : 32 * c;
-          uint32_t gr[32], ur[32];
-          tmem_ld_32x32b_x32(taddr + g * 128 + off, gr);
-          tmem_ld_32x32b_x32(taddr + g * 128 + 64 + off, ur);
+        for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, g);
+          tmem_ld_32x32b_x32(taddr + 128 + ch * 32, u);
           tmem_ld_wait();
-          const int col0 = ti.n_blk * 128 + (ti.half ? 64 * (sub >> 1) : 64 * g) + off;
+          const int col0 = ti.n_blk * 128 + ch * 32;
           if (col0 >= I) continue;  // warp-uniform
           float v[32];
           if (p.out != nullptr) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(gr[j])) * __uint_as_float(ur[j]);
+            for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(g[j])) * __uint_as_float(u[j]);
             emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, I, wrows, tr_row, tr_q, lane);
           }
           if (p.gu != nullptr) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(gr[j]);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(g[j]);
             emit_chunk(stg, v, p.gu, wrow0, 2 * I, col0, I, wrows, tr_row, tr_q, lane);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ur[j]);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
             emit_chunk(stg, v, p.gu + I, wrow0, 2 * I, col0, I, wrows, tr_row, tr_q, lane);
           }
         }
@@ -639,10 +604,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) wrow[i] = __shfl_sync(0xffffffffu, wq, i * 8 + tr_row);
 #pragma unroll 1
-        for (int ch = ch0; ch < ch0 + nch; ++ch) {
-          const int col = ti.n_blk * kBN + col_base + ch * 32 + tr_q * 8;
+        for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
+          const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
           uint4 nxt[12];
-          if (ch + 1 < ch0 + nch) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
+          if (ch + 1 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
           uint32_t a[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
@@ -679,36 +644,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
         }
-        // Each row's partial dot product is spread over the 4 lanes with the
-        // same l/4. Slots per (row, N tile): 4; full tile: warp half h writes
-        // slot 2h and zeroes 2h+1; half tile: slot 2*(sub>>1) + h.
+        // each row's partial dot product is spread over the 4 lanes with the
+        // same l/4; the two column halves write separate slots
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 1);
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 2);
           const int r = i * 8 + tr_row;
-          if (tr_q == 0 && r < wrows) {
-            float* slot = p.dw_part + (wrow0 + r) * (4 * p.n_tiles) + 4 * ti.n_blk;
-            if (ti.half) {
-              slot[2 * (sub >> 1) + half_w] = dwp[i];
-            } else {
-              slot[2 * half_w] = dwp[i];
-              slot[2 * half_w + 1] = 0.0f;
-            }
-            if (kEpiWarps == 4 && !ti.half) {
-              slot[2] = 0.0f;
-              slot[3] = 0.0f;
-            }
-          }
+          if (tr_q == 0 && r < wrows)
+            p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
+          if (kEpiWarps == 4 && tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + 1] = 0.f;
         }
       } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
 #pragma unroll 1
-        for (int ch = ch0; ch < ch0 + nch; ch += 2) {
+        for (int ch = ch0; ch < ch0 + kChunks; ch += 2) {
           uint32_t a0[32], a1[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a0);
           tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, a1);
           tmem_ld_wait();
-          const int col0 = ti.n_blk * kBN + col_base + ch * 32;
+          const int col0 = ti.n_blk * kBN + ch * 32;
           float v[32];
           if (col0 < p.N) {  // warp-uniform
 #pragma unroll

@@ -235,7 +235,7 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
   L.dGU = off; off += round256(P * 2 * I * 2);
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
-  L.dw_part = off; off += round256(P * 4 * cdiv(I, kBN) * 4);
+  L.dw_part = off; off += round256(P * 2 * cdiv(I, kBN) * 4);
   L.maps = off; off += round256(static_cast<size_t>(4) * E * sizeof(CUtensorMap));
   L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
   L.total = off;
@@ -402,7 +402,7 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   if (int st = current_device_info(&dev)) return st;
 
   GemmParams gu = base_params(E, P, offsets);
-  if (!make_map(&gu.tmA, Xp, H, P, 64, 128) || !make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 64))
+  if (!make_map(&gu.tmA, Xp, H, P, 64, 128) || !make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
     return MOE_ERR_CUDA;
   gu.sorted_pair = sorted_pair;
   gu.N = I;
@@ -494,7 +494,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     moe_bf16* gu_ws = reinterpret_cast<moe_bf16*>(w8 + L.gu);
     GemmParams rc = base_params(E, P, offsets);
     if (!make_map(&rc.tmA, Xp, H, P, 64, 128) ||
-        !make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 64))
+        !make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
       return MOE_ERR_CUDA;
     rc.sorted_pair = sorted_pair;
     rc.N = I;
@@ -597,7 +597,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     int blocks = (T + 7) / 8;
     if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
     router_bwd_kernel<<<blocks, 256, sizeof(float) * 8 * E, stream>>>(probs, topk_idx, topk_w, dw_part, pair_pos,
-                                                                       4 * nt_dgrad_down, T, E, k, dlogits);
+                                                                       2 * nt_dgrad_down, T, E, k, dlogits);
     if (launch_status()) return MOE_ERR_CUDA;
   }
   return MOE_OK;

@@ -14,6 +14,8 @@ namespace moe {
 template <int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ O, const int32_t* __restrict__ pair_pos,
                                                       int64_t T, int k, int vec_per_row, uint4* __restrict__ Y) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t P = T * k;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 __global__ void __launch_bounds__(256) combine_kernel_any_k(const uint4* __restrict__ O,
                                                             const int32_t* __restrict__ pair_pos, int64_t T, int k,
                                                             int vec_per_row, uint4* __restrict__ Y) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t P = T * k;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -94,15 +98,11 @@ inline cudaError_t launch_combine(const void* O, const int32_t* pair_pos, int T,
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   const uint4* o = static_cast<const uint4*>(O);
   uint4* y = static_cast<uint4*>(Y);
-  if (k <= 4)
-    combine_kernel<4><<<blocks, 256, 0, s>>>(o, pair_pos, T, k, vec, y);
-  else if (k <= 8)
-    combine_kernel<8><<<blocks, 256, 0, s>>>(o, pair_pos, T, k, vec, y);
-  else if (k <= 16)
-    combine_kernel<16><<<blocks, 256, 0, s>>>(o, pair_pos, T, k, vec, y);
-  else
-    combine_kernel_any_k<<<blocks, 256, 0, s>>>(o, pair_pos, T, k, vec, y);
-  return cudaGetLastError();
+  const int64_t T64 = T;
+  if (k <= 4) return launch_pdl(combine_kernel<4>, dim3(blocks), dim3(256), 0, s, o, pair_pos, T64, k, vec, y);
+  if (k <= 8) return launch_pdl(combine_kernel<8>, dim3(blocks), dim3(256), 0, s, o, pair_pos, T64, k, vec, y);
+  if (k <= 16) return launch_pdl(combine_kernel<16>, dim3(blocks), dim3(256), 0, s, o, pair_pos, T64, k, vec, y);
+  return launch_pdl(combine_kernel_any_k, dim3(blocks), dim3(256), 0, s, o, pair_pos, T64, k, vec, y);
 }
 
 }  // namespace moe

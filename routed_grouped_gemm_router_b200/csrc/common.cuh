@@ -1,10 +1,12 @@
 // Shared device helpers: the device status word, bf16 packing, warp utilities.
 #pragma once
 #include <cstdint>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/moe.h"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -49,6 +51,28 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
     if (lane >= o) v += n;
   }
   return v;
+}
+
+// Launches `kernel` on stream `s` with programmatic stream serialisation, so
+// its set-up may overlap the tail of the previous kernel on the stream (the
+// kernel itself waits for that kernel's results, see griddep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+  attr[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

@@ -312,6 +312,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(s_tmem, kTmemCols);
     tmem_relinquish_pair();
   }
+  // everything above touches no global memory; from here on this kernel reads
+  // its predecessors' results
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
   __syncthreads();
   if (warp == 0 && !kWgrad) {
@@ -701,6 +705,8 @@ __global__ void __launch_bounds__(256) build_expert_maps_kernel(const __grid_con
                                                                 const int32_t* __restrict__ offsets, int E,
                                                                 CUtensorMap* __restrict__ out) {
   __shared__ alignas(128) CUtensorMap s_map[8];
+  griddep_wait();
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * 8 + warp;
   if (m >= 2 * E) return;  // warp-uniform

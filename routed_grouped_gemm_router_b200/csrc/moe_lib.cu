@@ -193,7 +193,8 @@ int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
   ProfScope ps(slot, s);
-  grouped_gemm_kernel<KIND><<<grid, kGemmThreads, smem, s>>>(p);
+  if (launch_pdl(grouped_gemm_kernel<KIND>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return launch_status();
 }
 
@@ -313,27 +314,31 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
   const size_t hist_smem = sizeof(int) * kPermWarps * E;
   {
     ProfScope ps(kProfPermCount, stream);
-    permute_count_kernel<<<nchunks, kPermThreads, hist_smem, stream>>>(topk_idx, P, E, chunk_hist);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kPermThreads), hist_smem, stream, topk_idx, P, E,
+                   chunk_hist) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   {
     ProfScope ps(kProfPermScan, stream);
-    permute_scan_kernel<<<1, 1024, 0, stream>>>(chunk_hist, nchunks, E, counts, offsets);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, chunk_hist, nchunks, E, counts, offsets) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   {
     ProfScope ps(kProfPermScatter, stream);
-    permute_scatter_kernel<<<nchunks, kPermThreads, hist_smem, stream>>>(topk_idx, P, E, chunk_hist, offsets,
-                                                                         sorted_pair, pair_pos);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(kPermThreads), hist_smem, stream, topk_idx, P, E,
+                   static_cast<const int*>(chunk_hist), static_cast<const int32_t*>(offsets), sorted_pair,
+                   pair_pos) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   if (gather) {
     ProfScope ps(kProfGatherX, stream);
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
-    gather_rows_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X), sorted_pair, P, k, H / 8,
-                                                   reinterpret_cast<uint4*>(Xp));
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(X),
+                   static_cast<const int32_t*>(sorted_pair), P, k, H / 8, reinterpret_cast<uint4*>(Xp)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }
@@ -484,9 +489,10 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     ProfScope ps(kProfGatherDy, stream);
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
-    gather_rows_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(dY), sorted_pair, P, k, H / 8,
-                                                   reinterpret_cast<uint4*>(dYp));
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(dY),
+                   static_cast<const int32_t*>(sorted_pair), P, k, H / 8, reinterpret_cast<uint4*>(dYp)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   // 2. g|u when the forward did not keep them
   const moe_bf16* gu = gu_save;
@@ -560,8 +566,9 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   {
     GemmParams wg = base_params(E, P, offsets);
     if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64) || !make_map(&wg.tmB, Xp, H, P, 64, 64)) return MOE_ERR_CUDA;
-    build_expert_maps_kernel<<<cdiv(2 * E, 8), 256, 0, stream>>>(wg.tmA, wg.tmB, offsets, E, maps);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wg.tmA, wg.tmB, offsets, E,
+                   maps) != cudaSuccess)
+      return MOE_ERR_CUDA;
     wg.expert_maps = maps;
     wg.M = 2 * I;
     wg.N = H;
@@ -577,8 +584,9 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   {
     GemmParams wd = base_params(E, P, offsets);
     if (!make_map(&wd.tmA, dYp, H, P, 64, 64) || !make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
-    build_expert_maps_kernel<<<cdiv(2 * E, 8), 256, 0, stream>>>(wd.tmA, wd.tmB, offsets, E, maps + 2 * E);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wd.tmA, wd.tmB, offsets, E,
+                   maps + 2 * E) != cudaSuccess)
+      return MOE_ERR_CUDA;
     wd.expert_maps = maps + 2 * E;
     wd.M = H;
     wd.N = I;
@@ -596,9 +604,10 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     ProfScope ps(kProfRouterBwd, stream);
     int blocks = (T + 7) / 8;
     if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
-    router_bwd_kernel<<<blocks, 256, sizeof(float) * 8 * E, stream>>>(probs, topk_idx, topk_w, dw_part, pair_pos,
-                                                                       2 * nt_dgrad_down, T, E, k, dlogits);
-    if (launch_status()) return MOE_ERR_CUDA;
+    if (launch_pdl(router_bwd_kernel, dim3(blocks), dim3(256), sizeof(float) * 8 * E, stream, probs, topk_idx, topk_w,
+                   static_cast<const float*>(dw_part), pair_pos, 4 * nt_dgrad_down, static_cast<int64_t>(T), E, k,
+                   dlogits) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }

@@ -52,6 +52,8 @@ __device__ __forceinline__ void warp_count_slice(const int32_t* __restrict__ fla
 
 __global__ void __launch_bounds__(kPermThreads) permute_count_kernel(const int32_t* __restrict__ flat, int64_t P,
                                                                      int E, int* __restrict__ chunk_hist) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int s_hist[];  // [kPermWarps][E]
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
@@ -73,6 +75,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_count_kernel(const int32
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int* __restrict__ chunk_hist, int nchunks, int E,
                                                             int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int s_warp[32];
   const int e = threadIdx.x;
   int total = 0;
@@ -111,6 +115,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
                                                                        const int32_t* __restrict__ offsets,
                                                                        int32_t* __restrict__ sorted_pair,
                                                                        int32_t* __restrict__ pair_pos) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int s_hist[];  // [kPermWarps][E] -> per-warp running bases
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
@@ -156,6 +162,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ X,
                                                           const int32_t* __restrict__ sorted_pair, int64_t P,
                                                           int k, int vec_per_row, uint4* __restrict__ Xp) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {

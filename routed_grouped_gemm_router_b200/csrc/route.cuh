@@ -17,6 +17,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                                     float* __restrict__ probs) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
@@ -125,8 +127,7 @@ inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_
   const int vpl = (E + 31) / 32;
 #define MOE_ROUTE_CASE(V)                                                                    \
   if (vpl <= V) {                                                                            \
-    route_kernel<V><<<blocks, threads, 0, s>>>(logits, T, E, k, idx, w, probs);             \
-    return cudaGetLastError();                                                               \
+    return launch_pdl(route_kernel<V>, dim3(blocks), dim3(threads), 0, s, logits, T, E, k, idx, w, probs); \
   }
   MOE_ROUTE_CASE(1)
   MOE_ROUTE_CASE(2)

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict
                                                          const float* __restrict__ dw_part,
                                                          const int32_t* __restrict__ pair_pos, int n_parts,
                                                          int64_t T, int E, int k, float* __restrict__ dlogits) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float s_row[];  // [8 warps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* row = s_row + warp * E;

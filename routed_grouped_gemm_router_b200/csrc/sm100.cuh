@@ -66,6 +66,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels of this library are launched with programmatic stream
+// serialisation: a kernel may start while its predecessor on the stream is
+// still finishing, so every kernel calls griddep_wait() before its first
+// global-memory access (it returns once the predecessor grid has completed
+// and its writes are visible), then griddep_launch_dependents() to let the
+// next kernel begin its own set-up.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -85,6 +85,10 @@ constexpr int kNumBarriers = 2 * kStages + 5;
 // which keeps both the row-wise writes (8 rows per quarter-warp phase) and
 // the transposed reads (2 rows x 4 pieces per phase) free of bank conflicts.
 constexpr int kStageStrideBytes = 64;
+// dgrad-down writes this many partial routing-weight sums per (row, N tile):
+// one per column half of the tile. The workspace layout and the router
+// backward read the same constant.
+constexpr int kDwSlotsPerNTile = 2;
 constexpr int kStageWarpBytes = 32 * kStageStrideBytes;
 
 struct GemmParams {
@@ -109,7 +113,7 @@ struct GemmParams {
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
   const uint16_t* h_in;       // BwdDgradDown: h
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
-  float* dw_part;             // BwdDgradDown: [P, 2 * n_tiles] partial routing-weight grads
+  float* dw_part;             // BwdDgradDown: [P, kDwSlotsPerNTile * n_tiles] partial routing-weight grads
 };
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
@@ -656,8 +660,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           dwp[i] += __shfl_xor_sync(0xffffffffu, dwp[i], 2);
           const int r = i * 8 + tr_row;
           if (tr_q == 0 && r < wrows)
-            p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + half] = dwp[i];
-          if (kEpiWarps == 4 && tr_q == 0 && r < wrows) p.dw_part[(wrow0 + r) * (2 * p.n_tiles) + 2 * ti.n_blk + 1] = 0.f;
+            p.dw_part[(wrow0 + r) * (kDwSlotsPerNTile * p.n_tiles) + kDwSlotsPerNTile * ti.n_blk + half] = dwp[i];
+          if (kEpiWarps == 4 && tr_q == 0 && r < wrows)
+            p.dw_part[(wrow0 + r) * (kDwSlotsPerNTile * p.n_tiles) + kDwSlotsPerNTile * ti.n_blk + 1] = 0.f;
         }
       } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
 #pragma unroll 1

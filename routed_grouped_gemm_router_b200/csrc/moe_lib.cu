@@ -236,7 +236,7 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
   L.dGU = off; off += round256(P * 2 * I * 2);
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
-  L.dw_part = off; off += round256(P * 2 * cdiv(I, kBN) * 4);
+  L.dw_part = off; off += round256(P * kDwSlotsPerNTile * cdiv(I, kBN) * 4);
   L.maps = off; off += round256(static_cast<size_t>(4) * E * sizeof(CUtensorMap));
   L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
   L.total = off;
@@ -605,7 +605,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     int blocks = (T + 7) / 8;
     if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
     if (launch_pdl(router_bwd_kernel, dim3(blocks), dim3(256), sizeof(float) * 8 * E, stream, probs, topk_idx, topk_w,
-                   static_cast<const float*>(dw_part), pair_pos, 4 * nt_dgrad_down, static_cast<int64_t>(T), E, k,
+                   static_cast<const float*>(dw_part), pair_pos, kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k,
                    dlogits) != cudaSuccess)
       return MOE_ERR_CUDA;
   }

@@ -28,6 +28,8 @@ def test_wait_that_runs_out_reports_timeout_and_context_survives():
     st_, grads = U.run_layer(inp, 2)
     fwd, bwd = U.oracle_full(inp, 2)
     U.assert_rel(U.to_np(st_.Y), fwd["Y"], "Y")
+    for name in ("dX", "dW_gu", "dW_d", "dlogits"):
+        U.assert_rel(U.to_np(grads[name]), bwd[name], name)
 
 
 def test_selftest_rejects_bad_limits():

@@ -336,7 +336,7 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
     if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(X),
-                   static_cast<const int32_t*>(sorted_pair), P, k, H / 8, reinterpret_cast<uint4*>(Xp)) !=
+                   static_cast<const int32_t*>(pair_pos), P, k, H / 8, reinterpret_cast<uint4*>(Xp)) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
   }
@@ -490,7 +490,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
     if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(dY),
-                   static_cast<const int32_t*>(sorted_pair), P, k, H / 8, reinterpret_cast<uint4*>(dYp)) !=
+                   static_cast<const int32_t*>(pair_pos), P, k, H / 8, reinterpret_cast<uint4*>(dYp)) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
   }

@@ -16,7 +16,7 @@
 //  3. scatter : each block recounts its chunk, derives per-warp bases and
 //               writes every pair at base + (rank among equal ids before it),
 //               so pairs of one expert keep ascending pair-id order.
-//  4. gather  : Xp[r] = X[sorted_pair[r] / k] with 16-byte vector copies.
+//  4. gather  : Xp[pair_pos[q]] = X[q / k] in pair order, 16-byte vectors.
 #pragma once
 #include "common.cuh"
 
@@ -156,21 +156,24 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
   }
 }
 
-// Xp[r, :] = X[sorted_pair[r] / k, :]; one warp per row, 16-byte vectors,
-// four loads in flight per lane. Rows whose pair id is out of range (only
-// possible after an invalid expert id was reported) are skipped.
+// Xp[pair_pos[q], :] = X[q / k, :] for every pair q: the rows are visited in
+// pair order, so the k copies of a token row are made by consecutive warps
+// while the row is in L1/L2 and every row of X is read from DRAM once even
+// when X is larger than L2. One warp per pair, 16-byte vectors, four loads in
+// flight per lane. Pairs whose row is out of range (only possible after an
+// invalid expert id was reported) are skipped.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ X,
-                                                          const int32_t* __restrict__ sorted_pair, int64_t P,
+                                                          const int32_t* __restrict__ pair_pos, int64_t P,
                                                           int k, int vec_per_row, uint4* __restrict__ Xp) {
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
-    const int32_t q = sorted_pair[r];
-    if (q < 0 || q >= P) continue;
-    const uint4* src = X + static_cast<int64_t>(q / k) * vec_per_row;
-    uint4* dst = Xp + r * vec_per_row;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); q < P; q += warps) {
+    const int32_t r = pair_pos[q];
+    if (r < 0 || r >= P) continue;
+    const uint4* src = X + (q / k) * vec_per_row;
+    uint4* dst = Xp + static_cast<int64_t>(r) * vec_per_row;
     for (int c0 = 0; c0 < vec_per_row; c0 += 128) {
       uint4 v[4];
 #pragma unroll

@@ -187,9 +187,11 @@ size_t moe_layer_bwd_workspace_bytes(int T, int E, int k, int H, int I, int reco
  *   dlogits   = softmax Jacobian of (renormalisation Jacobian of dw)
  * Experts with no rows get exactly zero dW.
  *
- * dY [T,H] bf16 in. Xp, h, offsets, sorted_pair, pair_pos, topk_idx, topk_w
+ * dY [T,H] bf16 in. Xp, offsets, sorted_pair, pair_pos, topk_idx, topk_w
  * and probs as produced by the forward calls. gu_save [P,2I] from
  * moe_experts_fwd, or NULL to recompute it (needs recompute_gu workspace).
+ * h is not read (h = silu(g)*u is recomputed from g|u in the dgrad epilogue,
+ * which saves its DRAM traffic); it may be NULL.
  * Outputs: dX [T,H] bf16, dW_gu [E,2I,H] bf16, dW_d [E,H,I] bf16,
  * dlogits [T,E] fp32. ws >= moe_layer_bwd_workspace_bytes(...).
  */

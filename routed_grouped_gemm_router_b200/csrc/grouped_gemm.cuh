@@ -26,8 +26,9 @@
 //              (odd CTA) of W_gu[e]; epilogue h = silu(g) * u.
 //  FwdDown     A = h[P,I], B = W_d[e][H,I], epilogue O = w_q * acc.
 //  BwdDgradDown   A = dYp[P,H], B = W_d[e] read MN-major ([H,I] as K x N);
-//              epilogue: partial dw = <acc, h>, dh = w_q*acc, SwiGLU backward
-//              -> dGU = [dg | du], and hw = w_q * h for the down wgrad.
+//              epilogue: h = silu(g) * u from the saved g|u, partial
+//              dw = <acc, h>, dh = w_q*acc, SwiGLU backward -> dGU = [dg | du],
+//              and hw = w_q * h for the down wgrad.
 //  BwdDgradGateUp A = dGU[P,2I], B = W_gu[e] MN-major ([2I,H] as K x N) -> dXp.
 //  BwdWgrad    per expert dW[e] = A^T B with the expert's rows as K; both
 //              operands MN-major, loaded through per-expert tensor maps whose
@@ -111,7 +112,6 @@ struct GemmParams {
   int64_t out_ld;
   int64_t out_expert_stride;  // wgrad: elements per expert
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
-  const uint16_t* h_in;       // BwdDgradDown: h
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
   float* dw_part;             // BwdDgradDown: [P, kDwSlotsPerNTile * n_tiles] partial routing-weight grads
 };
@@ -235,21 +235,21 @@ __device__ __forceinline__ void emit_chunk(uint8_t* stg, const float (&v)[32], u
 }
 
 // dgrad-down epilogue operands in the transposed domain: for rows 8*i + tr_row
-// of the warp, 8 columns from `col`: g, u and h (16 bytes each); zeros for
-// rows or columns that do not exist.
+// of the warp, 8 columns from `col`: g and u (16 bytes each); zeros for rows
+// or columns that do not exist. (h is recomputed as silu(g) * u, which saves a
+// third of the epilogue's loads; the loads, not the math, bound this kernel.)
 __device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t wrow0, int wrows, int col, int tr_row,
-                                                uint4 (&b)[12]) {
+                                                uint4 (&b)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = i * 8 + tr_row;
     if (r < wrows && col < p.I) {
       const int64_t gr = wrow0 + r;
       // (streaming-hint loads measured 16% slower here)
-      b[3 * i] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + col));
-      b[3 * i + 1] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + p.I + col));
-      b[3 * i + 2] = __ldg(reinterpret_cast<const uint4*>(p.h_in + gr * p.I + col));
+      b[2 * i] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + col));
+      b[2 * i + 1] = __ldg(reinterpret_cast<const uint4*>(p.gu + gr * (2 * p.I) + p.I + col));
     } else {
-      b[3 * i] = b[3 * i + 1] = b[3 * i + 2] = make_uint4(0, 0, 0, 0);
+      b[2 * i] = b[2 * i + 1] = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -567,9 +567,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       // dgrad-down: issue the first chunk's g/u/h loads before the wait so
       // their latency hides behind the main loop
-      uint4 dd_cur[12];
-      if constexpr (KIND == kBwdDgradDown)
+      // g/u of the first two chunks are requested before the wait; each later
+      // chunk two chunks ahead of its use
+      uint4 dd_cur[8], dd_nxt[8];
+      if constexpr (KIND == kBwdDgradDown) {
         dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + ch0 * 32 + tr_q * 8, tr_row, dd_cur);
+        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + (ch0 + 1) * 32 + tr_q * 8, tr_row, dd_nxt);
+      }
 
       const int acc = tcount & 1;
       if (!warp_wait(&tfull_bar[acc], (tcount >> 1) & 1)) {
@@ -614,8 +618,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
         for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
           const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
-          uint4 nxt[12];
-          if (ch + 1 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, nxt);
+          uint4 nxt2[8];
+          if (ch + 2 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 64, tr_row, nxt2);
           uint32_t a[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
@@ -628,19 +632,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int i = 0; i < 4; ++i) {
             const int r = i * 8 + tr_row;
             if (r < wrows && col < I) {
-              float dhp[8], gv[8], uv[8], hv[8], dg[8], du[8], hw[8];
+              float dhp[8], gv[8], uv[8], dg[8], du[8], hw[8];
               unpack8(read_piece(stg, r, tr_q), dhp);
-              unpack8(dd_cur[3 * i], gv);
-              unpack8(dd_cur[3 * i + 1], uv);
-              unpack8(dd_cur[3 * i + 2], hv);
+              unpack8(dd_cur[2 * i], gv);
+              unpack8(dd_cur[2 * i + 1], uv);
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                dwp[i] += dhp[j] * hv[j];
-                const float dh = wrow[i] * dhp[j];
                 const float sg = sigmoid_f(gv[j]);
+                const float hv = gv[j] * sg * uv[j];  // h = silu(g) * u
+                dwp[i] += dhp[j] * hv;
+                const float dh = wrow[i] * dhp[j];
                 du[j] = dh * gv[j] * sg;
                 dg[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));
-                hw[j] = wrow[i] * hv[j];
+                hw[j] = wrow[i] * hv;
               }
               const int64_t gr = wrow0 + r;
               store8_bf16(p.out + gr * p.out_ld + col, dg);
@@ -650,7 +654,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           __syncwarp();
 #pragma unroll
-          for (int x = 0; x < 12; ++x) dd_cur[x] = nxt[x];
+          for (int x = 0; x < 8; ++x) {
+            dd_cur[x] = dd_nxt[x];
+            dd_nxt[x] = nxt2[x];
+          }
         }
         // each row's partial dot product is spread over the 4 lanes with the
         // same l/4; the two column halves write separate slots

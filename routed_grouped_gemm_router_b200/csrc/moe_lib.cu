@@ -459,10 +459,11 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
-  if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_ptr(h) || !ok_ptr(probs) ||
+  if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_opt(h) || !ok_ptr(probs) ||
                 !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(sorted_pair) || !ok_ptr(pair_pos) ||
                 !ok_ptr(W_gu) || !ok_ptr(W_d) || !ok_ptr(dX) || !ok_ptr(dlogits)))
     return MOE_ERR_INVALID_ARG;
+  (void)h;  // not read: the dgrad-down epilogue recomputes h = silu(g) * u from g|u
   const bool recompute = (gu_save == nullptr);
   const BwdLayout L = bwd_layout(T, E, k, H, I, recompute);
   if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
@@ -531,7 +532,6 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     bd.out = dGU;
     bd.out_ld = 2 * I;
     bd.gu = const_cast<moe_bf16*>(gu);
-    bd.h_in = h;
     bd.hw_out = hw;
     bd.dw_part = dw_part;
     if (int st = launch_gemm<kBwdDgradDown>(bd, rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms), stream,

@@ -144,3 +144,17 @@ def test_repeated_calls_are_deterministic():
     b, gb = U.run_layer(inp, k)
     assert torch.equal(a.Y, b.Y) and torch.equal(ga["dX"], gb["dX"])
     assert torch.equal(ga["dW_gu"], gb["dW_gu"]) and torch.equal(ga["dlogits"], gb["dlogits"])
+
+
+def test_backward_without_h():
+    """The backward recomputes h from g|u; passing no h gives the same gradients."""
+    from routed_grouped_gemm_router_b200 import binding as B
+    T, H, E, k, I = 600, 192, 10, 3, 160
+    inp = small_inputs(T, H, E, k, I, seed=31)
+    st, grads = U.run_layer(inp, k)
+    d = U.to_dev(inp)
+    p = st.perm
+    g2 = B.moe_layer_bwd(d["dY"], p["Xp"], st.gu, None, st.probs, st.topk_idx, st.topk_w, p["offsets"],
+                         p["sorted_pair"], p["pair_pos"], T, E, k, d["W_gu"], d["W_d"])
+    for name in ("dX", "dW_gu", "dW_d", "dlogits"):
+        assert torch.equal(g2[name], grads[name]), name

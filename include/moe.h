@@ -220,6 +220,10 @@ int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream);
  * moe_profile_kernel_name); MOE_ERR_INVALID_ARG for an unknown name.
  */
 int moe_profile_enable(int on);
+/* Restricts recording to kernel `name` until the next moe_profile_enable
+ * (NULL: every kernel), so that one kernel can be timed with the least
+ * disturbance of the launch stream. MOE_ERR_INVALID_ARG for an unknown name. */
+int moe_profile_only(const char* name);
 int moe_profile_read(const char* name, double* total_ms, int* launches);
 /* Name of kernel slot i (0-based), NULL past the last one. */
 const char* moe_profile_kernel_name(int i);

@@ -37,6 +37,7 @@ _SIGNATURES = {
     "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
     "moe_selftest_wait_timeout": (_c_int, [_c_int, _c_void]),
     "moe_profile_enable": (_c_int, [_c_int]),
+    "moe_profile_only": (_c_int, [ctypes.c_char_p]),
     "moe_profile_read": (_c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
     "moe_profile_kernel_name": (ctypes.c_char_p, [_c_int]),
 }
@@ -192,6 +193,11 @@ def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_p
 # --------------------------------------------------------------- profiling
 def profile_enable(on: bool = True):
     _check("moe_profile_enable", lib().moe_profile_enable(1 if on else 0))
+
+
+def profile_only(name: str | None):
+    """Record only kernel `name` (None: all) until the next profile_enable."""
+    _check("moe_profile_only", lib().moe_profile_only(None if name is None else name.encode()))
 
 
 def profile_kernel_names() -> list[str]:

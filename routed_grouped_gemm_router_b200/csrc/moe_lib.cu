@@ -142,6 +142,7 @@ const char* const kProfNames[kProfSlots] = {
 struct Profiler {
   std::mutex mu;
   bool on = false;
+  int only = -1;  // record only this slot (-1: every slot)
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> recs[kProfSlots];
   std::vector<cudaEvent_t> pool;
   cudaEvent_t take() {
@@ -173,7 +174,7 @@ struct ProfScope {
   cudaEvent_t end = nullptr;
   ProfScope(int slot_, cudaStream_t s_) : slot(slot_), s(s_) {
     std::lock_guard<std::mutex> lock(g_prof.mu);
-    if (!g_prof.on) return;
+    if (!g_prof.on || (g_prof.only >= 0 && g_prof.only != slot)) return;
     cudaEvent_t start = g_prof.take();
     end = g_prof.take();
     cudaEventRecord(start, s);
@@ -624,7 +625,23 @@ int moe_profile_enable(int on) {
   std::lock_guard<std::mutex> lock(g_prof.mu);
   g_prof.clear();
   g_prof.on = (on != 0);
+  g_prof.only = -1;
   return MOE_OK;
+}
+
+int moe_profile_only(const char* name) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (name == nullptr) {
+    g_prof.only = -1;
+    return MOE_OK;
+  }
+  for (int i = 0; i < kProfSlots; ++i) {
+    if (std::strcmp(name, kProfNames[i]) == 0) {
+      g_prof.only = i;
+      return MOE_OK;
+    }
+  }
+  return MOE_ERR_INVALID_ARG;
 }
 
 int moe_profile_read(const char* name, double* total_ms, int* launches) {

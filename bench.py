@@ -96,9 +96,8 @@ def measured_traffic(kernel, workload):
 
 
 class ClockSampler:
-    """SM clock, power and clock-event reasons sampled every 10 ms (NVML,
-    read-only) inside the timed window; nvidia-smi every 100 ms when NVML is
-    not importable."""
+    """SM clock, power and clock-event reasons sampled about every 2 ms
+    (NVML, read-only) inside the timed window."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -142,7 +141,7 @@ class ClockSampler:
                     self.rows.append((sm, mx, pw, rs))
                 except Exception:
                     pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def stop(self):
         self.stop_flag = True
@@ -154,7 +153,7 @@ class ClockSampler:
         reasons = sorted({n for r in self.rows for n, bit in self.REASONS.items() if r[3] & bit})
         return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(r[1] for r in self.rows),
                 "reasons": reasons, "samples": len(self.rows), "power_w_max": max(r[2] for r in self.rows),
-                "power_w_median": statistics.median([r[2] for r in self.rows]), "source": "NVML, 10 ms"}
+                "power_w_median": statistics.median([r[2] for r in self.rows]), "source": "NVML, ~2 ms"}
 
 
 def blas_threads():

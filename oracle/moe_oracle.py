@@ -10,7 +10,9 @@ Sources (page title, then the part of the page):
     training" (axolotl issue #3155), *Feature description*: the reference
     semantics are Hugging Face's for-loop over experts -- each expert takes the
     tokens routed to it, runs its MLP and adds the result back. The experts here
-    are SwiGLU without bias (the same thread: "changed to silu").
+    are SwiGLU without bias (the same thread: "changed to silu"). The router is
+    a Linear(H -> E) whose weight is [E, H] (the same thread, discussion of the
+    router's weight shape).
   * fused-MoE Triton project summary (sourcepulse), *How It Works* and
     *Highlighted Details*: softmax -> top-k routing, expert indexing by sorting
     inputs by expert, grouped GEMM over the sorted rows.
@@ -221,6 +223,23 @@ def layer_backward(fwd: dict, dY, X, W_gu, W_d, k: int) -> dict:
     dw = dw_flat.reshape(T, k)
     dlogits = router_backward(dw, fwd["w"], fwd["probs"], fwd["idx"])
     return dict(dX=dX, dW_gu=dW_gu, dW_d=dW_d, dlogits=dlogits, dw=dw)
+
+
+# ------------------------------------------------------------------ router Linear
+def router_logits(X, W_r) -> np.ndarray:
+    """logits = X W_r^T in float64. W_r [E, H] is the router's Linear(H -> E)
+    weight ("Integration of fused moe kernel (e.g., megablocks) for efficient
+    moe training", axolotl issue #3155, discussion of the router's weight
+    shape: [num_experts, hidden_size], or nn.Linear(hidden_size, num_experts))."""
+    return _f64(X) @ _f64(W_r).T
+
+
+def router_logits_backward(dlogits, X, W_r):
+    """Gradients of ``router_logits`` for upstream d logits [T, E]:
+    dW_r = dlogits^T X  [E, H], and the router's share of dX, dlogits W_r  [T, H]
+    (the layer's dX is the experts' dX plus this)."""
+    dl = _f64(dlogits)
+    return dl.T @ _f64(X), dl @ _f64(W_r)
 
 
 # ----------------------------------------------------------- sampled (large sizes)

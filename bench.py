@@ -59,6 +59,11 @@ def kernel_work(name, wl):
         "route": T * E * 4 * 2 + T * k * 8,
         "router_bwd": T * E * 4 * 2 + T * k * 12 + P * 8 * ((I + 255) // 256),
         "permute_count": P * 4, "permute_scan": E * 8, "permute_scatter": P * 12,
+        # router Linear: X (bf16) and W_r (fp32) read once, logits / dW_r / dX written once
+        "router_split_w": E * H * 4 + 3 * E * H * 2, "router_split_dlogits": T * E * 4 + 3 * T * E * 2,
+        "gemm_router_logits": T * H * 2 + E * H * 4 + T * E * 4,
+        "gemm_router_wgrad": T * H * 2 + T * E * 4 + E * H * 4, "router_sum_splits": 2 * E * H * 4,
+        "gemm_router_dgrad": T * E * 4 + E * H * 4 + 2 * T * H * 2,
     }
     return "hbm", float(nbytes.get(name, 0))
 
@@ -72,9 +77,30 @@ def read_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha():
+# Device-code files behind each kernel (the launch code in moe_lib.cu is not
+# part of a kernel's identity).
+_KERNEL_FILES = [
+    (("gemm_router_", "router_split_", "router_sum_"), ["router_linear.cuh"]),
+    (("gemm_",), ["grouped_gemm.cuh"]),
+    (("route",), ["route.cuh"]),
+    (("permute_", "gather_"), ["permute.cuh"]),
+    (("combine_",), ["combine.cuh"]),
+    (("router_bwd",), ["router_bwd.cuh"]),
+]
+
+
+def kernel_source_sha(kernel=None):
+    """Hash of the device code of `kernel` (its own file plus the shared
+    sm100.cuh / common.cuh), or of every source file when kernel is None."""
+    csrc = os.path.join(ROOT, "routed_grouped_gemm_router_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*")))
+    if kernel is not None:
+        for prefixes, own in _KERNEL_FILES:
+            if kernel.startswith(prefixes):
+                files = [os.path.join(csrc, f) for f in own + ["sm100.cuh", "common.cuh"]]
+                break
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "routed_grouped_gemm_router_b200", "csrc", "*"))):
+    for p in files:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -83,7 +109,7 @@ def kernel_source_sha():
 def measured_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary of the same kernel
     source; None when there is none or the sources changed since."""
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
         text = open(p).read()
         if (re.search(rf"^kernel: {re.escape(kernel)}$", text, re.M)
@@ -167,14 +193,17 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_step(inp_sub, k, backward):
+def oracle_step(inp_sub, k, backward, router=False):
     from oracle import moe_oracle as orc
-    fwd = orc.layer_forward(inp_sub.logits, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
+    logits = orc.router_logits(inp_sub.X, inp_sub.W_r) if router else inp_sub.logits
+    fwd = orc.layer_forward(logits, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
     if backward:
-        orc.layer_backward(fwd, inp_sub.dY, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
+        bwd = orc.layer_backward(fwd, inp_sub.dY, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
+        if router:
+            orc.router_logits_backward(bwd["dlogits"], inp_sub.X, inp_sub.W_r)
 
 
-def cpu_sample(inp, wl, target_s):
+def cpu_sample(inp, wl, target_s, router=False):
     """The first T_s tokens of the batch (all E experts), T_s sized so one
     oracle fwd+bwd takes about target_s seconds on the host cores."""
     import copy
@@ -187,12 +216,12 @@ def cpu_sample(inp, wl, target_s):
 
     ts = min(wl.T, 64)
     t0 = time.perf_counter()
-    oracle_step(sub(ts), wl.k, wl.backward)
+    oracle_step(sub(ts), wl.k, wl.backward, router)
     dt = time.perf_counter() - t0
     while ts < wl.T and dt < target_s / 4:
         ts = min(wl.T, ts * 4)
         t0 = time.perf_counter()
-        oracle_step(sub(ts), wl.k, wl.backward)
+        oracle_step(sub(ts), wl.k, wl.backward, router)
         dt = time.perf_counter() - t0
     return sub(ts), ts
 
@@ -225,13 +254,13 @@ def run_reference(args, wl, rank):
     if rank != 0:
         return
     inp = make_inputs(wl, seed=args.seed)
-    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s)
+    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s, router=args.router_linear)
     sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
     for _ in range(args.warmup):
-        oracle_step(sample, wl.k, wl.backward)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(sample, wl.k, wl.backward)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear)
     dt = (time.perf_counter() - t0) / args.steps
     value = step_flops(sub_wl) / dt / 1e12
     desc = f"first {ts} of {wl.T} tokens, all {wl.E} experts, {'fwd+bwd' if wl.backward else 'fwd'} in float64"
@@ -249,7 +278,9 @@ def run_reference(args, wl, rank):
 
 def workload_config(wl, args):
     return {"workload": f"{wl.name} MoE layer {'fwd+bwd' if wl.backward else 'fwd'}: T={wl.T} H={wl.H} "
-                        f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else ""),
+                        f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else "")
+                        + (" + router Linear (fp32, on the GPU)" if getattr(args, "router_linear", False) else ""),
+            "router_linear": bool(getattr(args, "router_linear", False)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -262,6 +293,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qwen3-30b-a3b", choices=sorted(WORKLOADS))
     ap.add_argument("--forward-only", action="store_true")
+    ap.add_argument("--router-linear", action="store_true",
+                    help="include the router Linear (logits = X W_r^T and its backward) in the step")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -297,12 +330,21 @@ def main():
     inp = make_inputs(wl, seed=args.seed + rank, with_dy=wl.backward)
     X, W_gu, W_d = inp.X.to(dev), inp.W_gu.to(dev), inp.W_d.to(dev)
     logits = inp.logits.to(dev)
+    W_r = inp.W_r.to(dev)
     dY = inp.dY.to(dev) if wl.backward else None
-    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True)
+    rl = args.router_linear
+    if rl and wl.zipf_s:
+        ap.error("--router-linear: the stress workloads' logit bias has no router-weight form")
+    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
+        if rl:
+            st = layer.forward_from_x(X, W_r, W_gu, W_d, wl.k, bufs=bufs)
+            if wl.backward:
+                layer.backward_to_x(st, dY, X, W_r, W_gu, W_d, bufs=bufs)
+            return
         st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs)
         if wl.backward:
             layer.backward(st, dY, W_gu, W_d, bufs=bufs)
@@ -380,7 +422,8 @@ def main():
         out_h = dict(Y=torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory(),
                      dX=torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory(),
                      dlogits=torch.empty(wl.T, wl.E, dtype=torch.float32).pin_memory())
-        h2d = pin["X"].numel() * 2 + pin["logits"].numel() * 4 + (pin["dY"].numel() * 2 if wl.backward else 0)
+        h2d = (pin["X"].numel() * 2 + (0 if rl else pin["logits"].numel() * 4)
+               + (pin["dY"].numel() * 2 if wl.backward else 0))
         d2h = out_h["Y"].numel() * 2 + ((out_h["dX"].numel() * 2 + out_h["dlogits"].numel() * 4)
                                         if wl.backward else 0)
         din = [dict(X=torch.empty_like(X), logits=torch.empty_like(logits),
@@ -401,7 +444,8 @@ def main():
             with torch.cuda.stream(up):
                 up.wait_event(ev_used[b])
                 din[b]["X"].copy_(pin["X"], non_blocking=True)
-                din[b]["logits"].copy_(pin["logits"], non_blocking=True)
+                if not rl:
+                    din[b]["logits"].copy_(pin["logits"], non_blocking=True)
                 if wl.backward:
                     din[b]["dY"].copy_(pin["dY"], non_blocking=True)
                 ev_in[b].record(up)
@@ -417,9 +461,14 @@ def main():
                     upload((i + 1) % 2)
                 stream.wait_event(ev_in[b])
                 stream.wait_event(ev_copied[b])
-                st = layer.forward(din[b]["logits"], din[b]["X"], W_gu, W_d, wl.k, bufs=obufs[b])
-                if wl.backward:
-                    g = layer.backward(st, din[b]["dY"], W_gu, W_d, bufs=obufs[b])
+                if rl:
+                    st = layer.forward_from_x(din[b]["X"], W_r, W_gu, W_d, wl.k, bufs=obufs[b])
+                    if wl.backward:
+                        g = layer.backward_to_x(st, din[b]["dY"], din[b]["X"], W_r, W_gu, W_d, bufs=obufs[b])
+                else:
+                    st = layer.forward(din[b]["logits"], din[b]["X"], W_gu, W_d, wl.k, bufs=obufs[b])
+                    if wl.backward:
+                        g = layer.backward(st, din[b]["dY"], W_gu, W_d, bufs=obufs[b])
                 ev_used[b].record(stream)
                 ev_out[b].record(stream)
                 with torch.cuda.stream(down):
@@ -489,9 +538,9 @@ def main():
 
     cpu = None
     if not args.no_cpu_baseline:
-        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s)
+        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl)
         t0 = time.perf_counter()
-        oracle_step(sample, wl.k, wl.backward)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear)
         dt = time.perf_counter() - t0
         sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
         cpu = {"value": step_flops(sub_wl) / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

@@ -202,6 +202,49 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Router Linear -- logits = X W_r^T and its backward, on the tensor cores.
+ * Source: "Integration of fused moe kernel (e.g., megablocks) for efficient
+ * moe training" (axolotl issue #3155), discussion of the router's weight
+ * shape: the router is a Linear(hidden -> experts) whose weight is
+ * [num_experts, hidden]; the router runs in fp32.
+ *
+ * X [T,H] is bf16, W_r [E,H] fp32. Every fp32 operand is split exactly into
+ * three bf16 terms on the device, so the logits are the exact products of X
+ * and W_r summed in fp32 (tensor-core accumulation order; split-K partial
+ * sums added in a fixed order, so results are deterministic).
+ * Limits: T >= 0, 3*T < 2^31, 1 <= E <= 1024, H a positive multiple of 8.
+ */
+
+/* Scratch bytes for moe_router_fwd and moe_router_bwd (the same buffer
+ * serves both); 0 for invalid shapes. */
+size_t moe_router_workspace_bytes(int T, int H, int E);
+
+/*
+ * moe_router_fwd -- logits = X W_r^T, then what moe_route computes from them.
+ *   logits [T,E] fp32 (optional output, may be NULL), topk_idx [T,k] int32,
+ *   topk_w [T,k] fp32, probs [T,E] fp32 (optional, may be NULL): the same
+ *   outputs, with the same rules, as moe_route applied to these logits.
+ *   ws >= moe_router_workspace_bytes(T, H, E).
+ */
+int moe_router_fwd(const moe_bf16* X, const float* W_r, int T, int H, int E, int k, float* logits,
+                   int32_t* topk_idx, float* topk_w, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_router_bwd -- gradients of logits = X W_r^T for upstream dlogits [T,E]
+ * fp32 (for instance moe_layer_bwd's output).
+ *   dW_r [E,H] fp32 (output, may be NULL): dlogits^T X, exact products of the
+ *     fp32 dlogits and bf16 X summed in fp32.
+ *   dX [T,H] bf16 (in/out, may be NULL): on entry the rest of the layer's
+ *     input gradient (moe_layer_bwd's dX); on return bf16(dX + dlogits W_r),
+ *     the product carried to about 2^-16 relative (the two leading bf16
+ *     terms of each operand), far below the bf16 rounding of the result.
+ *   X is read only for dW_r, W_r only for dX. With T == 0, dW_r is zeroed.
+ *   ws >= moe_router_workspace_bytes(T, H, E).
+ */
+int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, int T, int H, int E, float* dW_r,
+                   moe_bf16* dX, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_selftest_wait_timeout -- diagnostics: enqueues one kernel that waits on
  * a barrier nothing signals, using the same bounded wait as the pipeline
  * kernels but with a limit of limit_ms (1..2000) milliseconds. When the limit

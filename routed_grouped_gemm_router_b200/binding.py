@@ -35,6 +35,11 @@ _SIGNATURES = {
     "moe_combine": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void]),
     "moe_layer_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
+    "moe_router_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "moe_router_fwd": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void,
+                                _c_void, _c_void, _c_size, _c_void]),
+    "moe_router_bwd": (_c_int, [_c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void,
+                                _c_size, _c_void]),
     "moe_selftest_wait_timeout": (_c_int, [_c_int, _c_void]),
     "moe_profile_enable": (_c_int, [_c_int]),
     "moe_profile_only": (_c_int, [ctypes.c_char_p]),
@@ -188,6 +193,55 @@ def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_p
         _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]),
         _ptr(o["dW_gu"]), _ptr(o["dW_d"]), _ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream)))
     return o
+
+
+def _router_ws(T, H, E, dev, ws):
+    need = lib().moe_router_workspace_bytes(T, H, E)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    return ws
+
+
+def moe_router_fwd(X, W_r, k, out=None, want_logits=True, want_probs=True, ws=None, stream=None):
+    """logits = X W_r^T on the GPU, then routing; returns a dict with
+    logits, topk_idx, topk_w, probs (logits/probs None when not wanted)."""
+    T, H = X.shape
+    E = W_r.shape[0]
+    dev = X.device
+    _need(X, torch.bfloat16, (T, H), "X")
+    _need(W_r, torch.float32, (E, H), "W_r")
+    o = dict(out or {})
+    if want_logits:
+        o.setdefault("logits", torch.empty(T, E, dtype=torch.float32, device=dev))
+    if want_probs:
+        o.setdefault("probs", torch.empty(T, E, dtype=torch.float32, device=dev))
+    o.setdefault("topk_idx", torch.empty(T, k, dtype=torch.int32, device=dev))
+    o.setdefault("topk_w", torch.empty(T, k, dtype=torch.float32, device=dev))
+    ws = _router_ws(T, H, E, dev, ws)
+    _check("moe_router_fwd", lib().moe_router_fwd(
+        _ptr(X), _ptr(W_r), T, H, E, k, _ptr(o.get("logits")), _ptr(o["topk_idx"]), _ptr(o["topk_w"]),
+        _ptr(o.get("probs")), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_router_bwd(dlogits, X, W_r, dX=None, dW_r=None, want_dW_r=True, ws=None, stream=None):
+    """dW_r = dlogits^T X (fp32, allocated when not given and wanted) and, when
+    dX is given, dX += dlogits W_r in place. Returns (dW_r, dX)."""
+    T, E = dlogits.shape
+    H = W_r.shape[1]
+    dev = dlogits.device
+    _need(dlogits, torch.float32, (T, E), "dlogits")
+    _need(W_r, torch.float32, (E, H), "W_r")
+    _need(X, torch.bfloat16, (T, H), "X")
+    if dX is not None:
+        _need(dX, torch.bfloat16, (T, H), "dX")
+    if dW_r is None and want_dW_r:
+        dW_r = torch.empty(E, H, dtype=torch.float32, device=dev)
+    ws = _router_ws(T, H, E, dev, ws)
+    _check("moe_router_bwd", lib().moe_router_bwd(
+        _ptr(dlogits), _ptr(X), _ptr(W_r), T, H, E, _ptr(dW_r), _ptr(dX), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return dW_r, dX
 
 
 # --------------------------------------------------------------- profiling

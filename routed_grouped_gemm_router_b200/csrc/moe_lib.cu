@@ -21,6 +21,7 @@
 #include "permute.cuh"
 #include "route.cuh"
 #include "router_bwd.cuh"
+#include "router_linear.cuh"
 
 namespace moe {
 
@@ -100,12 +101,13 @@ EncodeTiledFn encode_fn() {
 
 // bf16 2-D row-major tensor [rows, inner], 128-byte swizzled boxes of
 // box_inner x box_rows; out-of-range elements read as zero.
+// row_stride_elems (0: = inner) is the distance between rows in elements.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
-              uint32_t box_rows) {
+              uint32_t box_rows, uint64_t row_stride_elems = 0) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {(row_stride_elems ? row_stride_elems : inner) * 2};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -131,13 +133,21 @@ enum ProfSlot : int {
   kProfWgradGateUp,
   kProfWgradDown,
   kProfRouterBwd,
+  kProfRouterSplitW,
+  kProfRouterLogits,
+  kProfRouterSplitDl,
+  kProfRouterWgrad,
+  kProfRouterSumSplits,
+  kProfRouterDgrad,
   kProfSlots
 };
 const char* const kProfNames[kProfSlots] = {
     "route",          "permute_count",       "permute_scan",           "permute_scatter",
     "gather_x",       "gemm_fwd_gate_up",    "gemm_fwd_down",          "combine_y",
     "gather_dy",      "gemm_recompute_gate_up", "gemm_bwd_dgrad_down", "gemm_bwd_dgrad_gate_up",
-    "combine_dx",     "gemm_bwd_wgrad_gate_up", "gemm_bwd_wgrad_down", "router_bwd"};
+    "combine_dx",     "gemm_bwd_wgrad_gate_up", "gemm_bwd_wgrad_down", "router_bwd",
+    "router_split_w", "gemm_router_logits",  "router_split_dlogits",   "gemm_router_wgrad",
+    "router_sum_splits", "gemm_router_dgrad"};
 
 struct Profiler {
   std::mutex mu;
@@ -242,6 +252,79 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
   L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
   L.total = off;
   return L;
+}
+
+// ------------------------------------------------------------ router Linear
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Workspace of moe_router_fwd / moe_router_bwd: the bf16 terms of W_r
+// [3E, H], those of dlogits [3T, E8] (rows padded to E8 = E rounded up to 8,
+// so that rows start on 16 bytes) and the fp32 split-K partials (at most
+// kRgMaxSplitsLogits x [T, E8] for the logits, kRgMaxSplitsWgrad x [E, H] for
+// dW_r).
+struct RouterLayout {
+  size_t w3, dl3, part, total;
+};
+RouterLayout router_layout(int T, int H, int E) {
+  const size_t E8 = static_cast<size_t>(round_up(E, 8));
+  RouterLayout L;
+  size_t off = 0;
+  L.w3 = off; off += round256(size_t(3) * E * H * 2);
+  L.dl3 = off; off += round256(size_t(3) * T * E8 * 2);
+  const size_t part_fwd = size_t(kRgMaxSplitsLogits) * T * E8 * 4;
+  const size_t part_bwd = size_t(kRgMaxSplitsWgrad) * E * H * 4;
+  L.part = off; off += round256(part_fwd > part_bwd ? part_fwd : part_bwd);
+  L.total = off;
+  return L;
+}
+
+bool router_shape_ok(int T, int H, int E) {
+  return T >= 0 && E >= 1 && E <= kMaxExperts && dims_ok(H) && 3 * static_cast<int64_t>(T) < (int64_t(1) << 31);
+}
+
+// CTAs of a router GEMM that fit on one SM (shared memory and TMEM).
+int router_residency(int bn, int stages) {
+  const size_t per = rg_smem_bytes(bn, stages) + 1024;  // + the per-CTA reservation
+  int r = static_cast<int>((228 * 1024) / per);
+  const int tmem = 512 / rg_tmem_cols(bn);
+  if (r > tmem) r = tmem;
+  return r < 1 ? 1 : r;
+}
+
+// Split-K count: enough units for every resident CTA slot of the device, at
+// most `cap`, never more splits than K blocks.
+int router_splits(int64_t tiles, int k_blocks, int cap, int slots) {
+  int64_t s = (slots + tiles - 1) / tiles;
+  if (s > cap) s = cap;
+  if (s > k_blocks) s = k_blocks;
+  return s < 1 ? 1 : static_cast<int>(s);
+}
+
+template <int KIND>
+int launch_router_gemm(const RouterGemmParams& p, cudaStream_t s, int slot) {
+  const size_t smem = rg_smem_bytes(p.bn, p.stages);
+  if (cudaFuncSetAttribute(router_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ProfScope ps(slot, s);
+  const int64_t grid = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.splits;
+  if (launch_pdl(router_gemm_kernel<KIND>, dim3(static_cast<unsigned>(grid)), dim3(kRgThreads), smem, s, p) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_status();
+}
+
+int launch_split3(const float* src, int64_t rows, int cols, int src_ld, int dst_ld, int64_t term_rows,
+                  uint16_t* dst, int num_sms, cudaStream_t s, int slot) {
+  const int64_t n = rows * cols;
+  if (n == 0) return MOE_OK;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > int64_t(num_sms) * 8) blocks = int64_t(num_sms) * 8;
+  ProfScope ps(slot, s);
+  if (launch_pdl(split3_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, src, rows, cols, src_ld,
+                 dst_ld, term_rows, dst) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_status();
 }
 
 }  // namespace
@@ -609,6 +692,131 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                    static_cast<const float*>(dw_part), pair_pos, kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k,
                    dlogits) != cudaSuccess)
       return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+size_t moe_router_workspace_bytes(int T, int H, int E) {
+  if (!router_shape_ok(T, H, E)) return 0;
+  return router_layout(T, H, E).total;
+}
+
+int moe_router_fwd(const moe_bf16* X, const float* W_r, int T, int H, int E, int k, float* logits,
+                   int32_t* topk_idx, float* topk_w, float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!router_shape_ok(T, H, E) || !shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ok_ptr(X) || !ok_ptr(W_r) || !ok_opt(logits) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_opt(probs))
+    return MOE_ERR_INVALID_ARG;
+  const RouterLayout L = router_layout(T, H, E);
+  if (ws_bytes < L.total || !ok_ptr(ws)) return MOE_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* w3 = reinterpret_cast<uint16_t*>(w + L.w3);
+  float* part = reinterpret_cast<float*>(w + L.part);
+  const int E8 = round_up(E, 8);
+  if (int st = launch_split3(W_r, E, H, H, H, E, w3, dev->num_sms, stream, kProfRouterSplitW)) return st;
+
+  RouterGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = T;
+  p.N = E;
+  p.bn = E < 256 ? round_up(E, 16) : 256;
+  p.stages = p.bn <= 128 ? 3 : 4;
+  p.m_tiles = cdiv(T, kRgBM);
+  p.n_tiles = cdiv(E, p.bn);
+  p.nkb = cdiv(H, kRgBK);
+  p.n_terms = 3;
+  p.term_rows_b = E;
+  p.splits = router_splits(int64_t(p.m_tiles) * p.n_tiles, 3 * p.nkb, kRgMaxSplitsLogits,
+                           dev->num_sms * router_residency(p.bn, p.stages));
+  p.out = part;
+  p.out_ld = E8;
+  p.out_split_stride = int64_t(T) * E8;
+  if (!make_map(&p.tmA, X, H, T, 64, kRgBM) || !make_map(&p.tmB, w3, H, 3 * int64_t(E), 64, p.bn))
+    return MOE_ERR_CUDA;
+  if (int st = launch_router_gemm<kRgLogits>(p, stream, kProfRouterLogits)) return st;
+  ProfScope ps(kProfRoute, stream);
+  if (launch_route(nullptr, T, E, k, topk_idx, topk_w, probs, stream, part, p.splits, E8, int64_t(T) * E8, logits) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_status();
+}
+
+int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, int T, int H, int E, float* dW_r,
+                   moe_bf16* dX, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!router_shape_ok(T, H, E)) return MOE_ERR_INVALID_ARG;
+  if (!ok_opt(dW_r) || !ok_opt(dX)) return MOE_ERR_INVALID_ARG;
+  if (dW_r == nullptr && dX == nullptr) return MOE_OK;
+  if (T > 0 && (!ok_ptr(dlogits) || (dW_r != nullptr && !ok_ptr(X)) || (dX != nullptr && !ok_ptr(W_r))))
+    return MOE_ERR_INVALID_ARG;
+  const RouterLayout L = router_layout(T, H, E);
+  if (T > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  if (T == 0) {  // no tokens: dW_r = 0, dX is empty
+    if (dW_r != nullptr && cudaMemsetAsync(dW_r, 0, sizeof(float) * size_t(E) * H, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* w3 = reinterpret_cast<uint16_t*>(w + L.w3);
+  uint16_t* dl3 = reinterpret_cast<uint16_t*>(w + L.dl3);
+  float* part = reinterpret_cast<float*>(w + L.part);
+  const int E8 = round_up(E, 8);
+  if (int st = launch_split3(dlogits, T, E, E, E8, T, dl3, dev->num_sms, stream, kProfRouterSplitDl)) return st;
+
+  if (dW_r != nullptr) {  // dW_r^T [H, E] = X^T dl, split over K = tokens
+    RouterGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = H;
+    p.N = E;
+    p.bn = E < 256 ? round_up(E, 64) : 256;
+    p.stages = p.bn <= 128 ? 3 : 4;
+    p.m_tiles = cdiv(H, kRgBM);
+    p.n_tiles = cdiv(E, p.bn);
+    p.nkb = cdiv(T, kRgBK);
+    p.n_terms = 3;
+    p.term_rows_b = T;
+    p.splits = router_splits(int64_t(p.m_tiles) * p.n_tiles, 3 * p.nkb, kRgMaxSplitsWgrad,
+                             dev->num_sms * router_residency(p.bn, p.stages));
+    p.out = p.splits > 1 ? part : dW_r;
+    p.out_ld = H;
+    p.out_split_stride = int64_t(E) * H;
+    if (!make_map(&p.tmA, X, H, T, 64, 64) || !make_map(&p.tmB, dl3, E, 3 * int64_t(T), 64, 64, E8))
+      return MOE_ERR_CUDA;
+    if (int st = launch_router_gemm<kRgWgrad>(p, stream, kProfRouterWgrad)) return st;
+    if (p.splits > 1) {
+      const int64_t n = int64_t(E) * H;
+      int64_t blocks = (n / 4 + 255) / 256;
+      if (blocks > int64_t(dev->num_sms) * 8) blocks = int64_t(dev->num_sms) * 8;
+      ProfScope ps(kProfRouterSumSplits, stream);
+      if (launch_pdl(sum_splits_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                     static_cast<const float*>(part), p.splits, n, n, dW_r) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (int st = launch_status()) return st;
+    }
+  }
+  if (dX != nullptr) {  // dX [T, H] += dl W_r over the term pairs (0,0), (0,1), (1,0)
+    if (int st = launch_split3(W_r, E, H, H, H, E, w3, dev->num_sms, stream, kProfRouterSplitW)) return st;
+    RouterGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = T;
+    p.N = H;
+    p.bn = 128;
+    p.stages = 3;
+    p.m_tiles = cdiv(T, kRgBM);
+    p.n_tiles = cdiv(H, p.bn);
+    p.nkb = cdiv(E, kRgBK);
+    p.n_terms = 3;
+    p.term_rows_a = T;
+    p.term_rows_b = E;
+    p.splits = 1;
+    p.dx = dX;
+    p.dx_ld = H;
+    if (!make_map(&p.tmA, dl3, E, 3 * int64_t(T), 64, kRgBM, E8) || !make_map(&p.tmB, w3, H, 3 * int64_t(E), 64, 64))
+      return MOE_ERR_CUDA;
+    if (int st = launch_router_gemm<kRgDgrad>(p, stream, kProfRouterDgrad)) return st;
   }
   return MOE_OK;
 }

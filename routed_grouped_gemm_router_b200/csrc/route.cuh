@@ -5,7 +5,10 @@
 // review comment: top-k scores are divided by their sum + 1e-20.
 //
 // Lane l holds experts e = l + 32*v (v < VPL) in registers, so the logits row
-// is read once, coalesced. Selection compares the fp32 logits themselves
+// is read once, coalesced. With n_part > 0 the logits are not read from
+// `logits` but summed from the router GEMM's split-K partials
+// (part[s * part_stride + t * part_ld + e], s = 0..n_part-1 in order) and
+// written to `logits_out` (if not null). Selection compares the fp32 logits themselves
 // (logit descending, lower expert index on ties), which makes the chosen set
 // and its order exactly reproducible on any processor given the same logits.
 #pragma once
@@ -16,19 +19,30 @@ namespace moe {
 template <int VPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                                                    float* __restrict__ probs) {
+                                                    float* __restrict__ probs, const float* __restrict__ part,
+                                                    int n_part, int part_ld, int64_t part_stride,
+                                                    float* __restrict__ logits_out) {
   griddep_wait();
   griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
-    const float* row = logits + static_cast<int64_t>(t) * E;
     float l[VPL];
     float m = -INFINITY;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
       const int e = lane + 32 * v;
-      l[v] = (e < E) ? __ldg(row + e) : -INFINITY;
+      if (e >= E) {
+        l[v] = -INFINITY;
+      } else if (n_part == 0) {
+        l[v] = __ldg(logits + static_cast<int64_t>(t) * E + e);
+      } else {
+        const float* pp = part + static_cast<int64_t>(t) * part_ld + e;
+        float acc = __ldg(pp);
+        for (int s = 1; s < n_part; ++s) acc += __ldg(pp + s * part_stride);
+        l[v] = acc;
+        if (logits_out != nullptr) logits_out[static_cast<int64_t>(t) * E + e] = acc;
+      }
       m = fmaxf(m, l[v]);
     }
     m = warp_max_f(m);
@@ -118,7 +132,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 
 // One-pass launch: picks the register width from E.
 inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* idx, float* w, float* probs,
-                                cudaStream_t s) {
+                                cudaStream_t s, const float* part = nullptr, int n_part = 0, int part_ld = 0,
+                                int64_t part_stride = 0, float* logits_out = nullptr) {
   if (T == 0) return cudaSuccess;
   const int threads = 256;
   const int warps = threads / 32;
@@ -127,7 +142,8 @@ inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_
   const int vpl = (E + 31) / 32;
 #define MOE_ROUTE_CASE(V)                                                                    \
   if (vpl <= V) {                                                                            \
-    return launch_pdl(route_kernel<V>, dim3(blocks), dim3(threads), 0, s, logits, T, E, k, idx, w, probs); \
+    return launch_pdl(route_kernel<V>, dim3(blocks), dim3(threads), 0, s, logits, T, E, k, idx, w, probs, part, \
+                      n_part, part_ld, part_stride, logits_out);                                                \
   }
   MOE_ROUTE_CASE(1)
   MOE_ROUTE_CASE(2)

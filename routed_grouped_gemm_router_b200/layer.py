@@ -1,8 +1,11 @@
-"""The whole expert layer as a sequence of the five C-ABI calls.
+"""The whole expert layer as a sequence of the C-ABI calls.
 
 ``forward`` runs moe_route -> moe_permute -> moe_experts_fwd -> moe_combine
-and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. All
-buffers are torch CUDA tensors; nothing here does arithmetic.
+and returns Y plus the saved state; ``backward`` runs moe_layer_bwd.
+``forward_from_x`` / ``backward_to_x`` also run the router Linear
+(moe_router_fwd in place of moe_route; moe_router_bwd after moe_layer_bwd,
+adding the router's share to dX and giving dW_r). All buffers are torch CUDA
+tensors; nothing here does arithmetic.
 """
 from __future__ import annotations
 
@@ -26,6 +29,7 @@ class LayerState:
     gu: torch.Tensor | None
     O: torch.Tensor
     Y: torch.Tensor
+    logits: torch.Tensor | None = None
 
 
 def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
@@ -35,6 +39,23 @@ def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torc
     b = bufs or {}
     T, E = logits.shape
     idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
+    return _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream)
+
+
+def forward_from_x(X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
+                   save_gu: bool = True, bufs: dict | None = None, stream=None) -> LayerState:
+    """As ``forward``, with the logits computed on the GPU from the fp32
+    router weight W_r [E, H] (moe_router_fwd)."""
+    b = bufs or {}
+    T, E = X.shape[0], W_r.shape[0]
+    out = {n: b[n] for n in ("logits", "topk_idx", "topk_w", "probs") if b.get(n) is not None}
+    r = B.moe_router_fwd(X, W_r, k, out=out, ws=b.get("router_ws"), stream=stream)
+    st = _experts_forward(T, E, k, r["topk_idx"], r["topk_w"], r["probs"], X, W_gu, W_d, save_gu, b, stream)
+    st.logits = r["logits"]
+    return st
+
+
+def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream) -> LayerState:
     perm = B.moe_permute(idx, E, X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
     h, gu, O = B.moe_experts_fwd(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k, W_gu, W_d,
                                  h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"), save_gu=save_gu,
@@ -53,7 +74,19 @@ def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Te
                            out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream)
 
 
-def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True) -> dict:
+def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor,
+                  W_d: torch.Tensor, bufs: dict | None = None, stream=None) -> dict:
+    """``backward`` plus the router Linear's: dX gains dlogits W_r (in place)
+    and the result holds dW_r = dlogits^T X."""
+    b = bufs or {}
+    g = backward(st, dY, W_gu, W_d, bufs=b, stream=stream)
+    dW_r, _ = B.moe_router_bwd(g["dlogits"], X, W_r, dX=g["dX"], dW_r=b.get("dW_r"), ws=b.get("router_ws"),
+                               stream=stream)
+    g["dW_r"] = dW_r
+    return g
+
+
+def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False) -> dict:
     """Every output and workspace of one forward+backward, allocated once."""
     P = T * k
     bf = torch.bfloat16
@@ -79,4 +112,9 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
         bwd_ws=torch.empty(max(lib.moe_layer_bwd_workspace_bytes(T, E, k, H, I, 0 if save_gu else 1), 1),
                            dtype=torch.uint8, device=device),
     )
+    if router:
+        d["logits"] = torch.empty(T, E, dtype=torch.float32, device=device)
+        d["dW_r"] = torch.empty(E, H, dtype=torch.float32, device=device)
+        d["router_ws"] = torch.empty(max(lib.moe_router_workspace_bytes(T, H, E), 1), dtype=torch.uint8,
+                                     device=device)
     return d

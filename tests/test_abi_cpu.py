@@ -72,3 +72,27 @@ def test_profile_names():
     names = B.profile_kernel_names()
     assert "gemm_fwd_gate_up" in names and "router_bwd" in names
     assert len(names) == len(set(names))
+
+
+def test_router_linear_arguments_rejected_without_device():
+    lib = B.lib()
+    p = ctypes.c_void_p(256)
+    odd = ctypes.c_void_p(264 + 2)
+    assert lib.moe_router_workspace_bytes(8192, 2048, 128) >= 3 * 128 * 2048 * 2 + 3 * 8192 * 128 * 2
+    assert lib.moe_router_workspace_bytes(8, 12, 4) == 0, "H must be a multiple of 8"
+    assert lib.moe_router_workspace_bytes(8, 16, 2000) == 0, "E > 1024"
+    need = lib.moe_router_workspace_bytes(16, 16, 4)
+    # forward: shapes, pointers, workspace
+    assert lib.moe_router_fwd(p, p, 16, 12, 4, 2, p, p, p, p, p, need, NULL) == 1   # H % 8
+    assert lib.moe_router_fwd(p, p, 16, 16, 4, 5, p, p, p, p, p, need, NULL) == 1   # k > E
+    assert lib.moe_router_fwd(NULL, p, 16, 16, 4, 2, p, p, p, p, p, need, NULL) == 1
+    assert lib.moe_router_fwd(p, odd, 16, 16, 4, 2, p, p, p, p, p, need, NULL) == 1
+    assert lib.moe_router_fwd(p, p, 16, 16, 4, 2, NULL, p, p, NULL, p, need - 1, NULL) == 3
+    assert lib.moe_router_fwd(p, p, 0, 16, 4, 2, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0  # empty batch
+    # backward
+    assert lib.moe_router_bwd(p, p, p, 16, 16, 4, NULL, NULL, NULL, 0, NULL) == 0      # nothing asked
+    assert lib.moe_router_bwd(NULL, p, p, 16, 16, 4, p, NULL, p, need, NULL) == 1      # no dlogits
+    assert lib.moe_router_bwd(p, NULL, p, 16, 16, 4, p, NULL, p, need, NULL) == 1      # dW_r needs X
+    assert lib.moe_router_bwd(p, p, NULL, 16, 16, 4, NULL, p, p, need, NULL) == 1      # dX needs W_r
+    assert lib.moe_router_bwd(p, p, p, 16, 16, 4, p, p, p, need - 1, NULL) == 3
+    assert "gemm_router_logits" in B.profile_kernel_names()

@@ -255,6 +255,7 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
 }
 
 // ------------------------------------------------------------ router Linear
+static_assert(kRgMaxSplitsLogits <= kRouteMaxParts, "the routing kernel sums at most kRouteMaxParts partials");
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Workspace of moe_router_fwd / moe_router_bwd: the bf16 terms of W_r
@@ -803,7 +804,7 @@ int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, in
     std::memset(&p, 0, sizeof(p));
     p.M = T;
     p.N = H;
-    p.bn = 128;
+    p.bn = kRgDgradBN;
     p.stages = 3;
     p.m_tiles = cdiv(T, kRgBM);
     p.n_tiles = cdiv(H, p.bn);

@@ -16,6 +16,9 @@
 
 namespace moe {
 
+// Most split-K partials of the router logits the routing kernel sums.
+constexpr int kRouteMaxParts = 8;
+
 template <int VPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
@@ -29,22 +32,56 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
     float l[VPL];
     float m = -INFINITY;
+    if (n_part == 0) {
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      const int e = lane + 32 * v;
-      if (e >= E) {
-        l[v] = -INFINITY;
-      } else if (n_part == 0) {
-        l[v] = __ldg(logits + static_cast<int64_t>(t) * E + e);
-      } else {
-        const float* pp = part + static_cast<int64_t>(t) * part_ld + e;
-        float acc = __ldg(pp);
-        for (int s = 1; s < n_part; ++s) acc += __ldg(pp + s * part_stride);
-        l[v] = acc;
-        if (logits_out != nullptr) logits_out[static_cast<int64_t>(t) * E + e] = acc;
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        l[v] = (e < E) ? __ldg(logits + static_cast<int64_t>(t) * E + e) : -INFINITY;
       }
-      m = fmaxf(m, l[v]);
+    } else if constexpr (VPL > 4) {
+      // wide rows: one partial at a time, the row's values in parallel
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) l[v] = 0.0f;
+      for (int s = 0; s < n_part; ++s) {
+        float pv[VPL];
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+          const int e = lane + 32 * v;
+          pv[v] = (e < E) ? __ldg(part + s * part_stride + static_cast<int64_t>(t) * part_ld + e) : 0.0f;
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) l[v] += pv[v];
+      }
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        if (e < E && logits_out != nullptr) logits_out[static_cast<int64_t>(t) * E + e] = l[v];
+        if (e >= E) l[v] = -INFINITY;
+      }
+    } else {
+      // every partial of every value is requested before the first add
+      float pv[kRouteMaxParts][VPL];
+#pragma unroll
+      for (int s = 0; s < kRouteMaxParts; ++s)
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+          const int e = lane + 32 * v;
+          pv[s][v] = (s < n_part && e < E) ? __ldg(part + s * part_stride + static_cast<int64_t>(t) * part_ld + e)
+                                           : 0.0f;
+        }
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        float acc = pv[0][v];
+#pragma unroll
+        for (int s = 1; s < kRouteMaxParts; ++s)
+          if (s < n_part) acc += pv[s][v];
+        l[v] = (e < E) ? acc : -INFINITY;
+        if (e < E && logits_out != nullptr) logits_out[static_cast<int64_t>(t) * E + e] = acc;
+      }
     }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) m = fmaxf(m, l[v]);
     m = warp_max_f(m);
     float z[VPL];
     float zsum = 0.f;

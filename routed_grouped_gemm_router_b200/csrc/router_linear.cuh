@@ -40,8 +40,9 @@ constexpr int kRgMaxStages = 4;
 constexpr int kRgThreads = 192;
 constexpr int kRgATileBytes = kRgBM * kRgBK * 2;  // 16 KiB
 constexpr int kRgStageWarpBytes = 32 * 128;       // 32 rows x 32 fp32 per epilogue warp
-constexpr int kRgMaxSplitsLogits = 8;
+constexpr int kRgMaxSplitsLogits = 8;  // the routing kernel sums at most 8 partials
 constexpr int kRgMaxSplitsWgrad = 32;
+constexpr int kRgDgradBN = 128;  // N tile of the dX part (its epilogue prefetch is sized for it)
 
 // (term of A, term of B) of the three products kept in the dX part.
 __host__ __device__ constexpr int rg_dgrad_term_a(int j) { return j == 2 ? 1 : 0; }
@@ -267,17 +268,64 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
     // row domain: for a fixed column the 32 lanes cover 32 consecutive floats.
     const int sub = warp & 3;
     uint8_t* stg = s_stage + (warp - 2) * kRgStageWarpBytes;
+    const int tr_row = lane >> 2;
+    const int tr_q = lane & 3;
+    // dX: the incoming values of this warp's rows are requested before the
+    // wait, so their DRAM latency overlaps the main loop
+    constexpr int kDxChunks = KIND == kRgDgrad ? kRgDgradBN / 32 : 1;
+    uint4 dxv[kDxChunks][4];
+    if constexpr (KIND == kRgDgrad) {
+#pragma unroll
+      for (int ch = 0; ch < kDxChunks; ++ch)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = m0 + sub * 32 + i * 8 + tr_row;
+          const int col = n0 + ch * 32 + tr_q * 8;
+          dxv[ch][i] = (row < p.M && col < p.N)
+                           ? *reinterpret_cast<const uint4*>(p.dx + static_cast<int64_t>(row) * p.dx_ld + col)
+                           : make_uint4(0, 0, 0, 0);
+        }
+    }
     const bool ok = rg_warp_wait(tfull_bar, 0);
     if (!ok) {
       if (lane == 0) report(MOE_ERR_TIMEOUT);
       *s_abort = 1;
     }
     tc_fence_after();
-    if (ok && !*s_abort) {
+    if (ok && !*s_abort && KIND == kRgDgrad) {
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
       const int row0 = m0 + sub * 32;
-      const int tr_row = lane >> 2;
-      const int tr_q = lane & 3;
+#pragma unroll
+      for (int ch = 0; ch < kDxChunks; ++ch) {
+        const int col0 = n0 + ch * 32;
+        if (col0 < p.N) {  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + ch * 32, v);
+          tmem_ld_wait();
+          rg_stage_row(stg, lane, v);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = row0 + i * 8 + tr_row;
+            const int col = col0 + tr_q * 8;
+            if (row < p.M && col < p.N) {  // N is a multiple of 8: bf16(dX + acc)
+              float f[8];
+              rg_read8(stg, i * 8 + tr_row, tr_q, f);
+              const uint4 old = dxv[ch][i];
+              uint4 o;
+              o.x = pack_bf16(bf16lo(old.x) + f[0], bf16hi(old.x) + f[1]);
+              o.y = pack_bf16(bf16lo(old.y) + f[2], bf16hi(old.y) + f[3]);
+              o.z = pack_bf16(bf16lo(old.z) + f[4], bf16hi(old.z) + f[5]);
+              o.w = pack_bf16(bf16lo(old.w) + f[6], bf16hi(old.w) + f[7]);
+              *reinterpret_cast<uint4*>(p.dx + static_cast<int64_t>(row) * p.dx_ld + col) = o;
+            }
+          }
+          __syncwarp();
+        }
+      }
+    } else if (ok && !*s_abort) {
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
+      const int row0 = m0 + sub * 32;
 #pragma unroll 1
       // TMEM holds rg_tmem_cols(bn) >= 32 * ceil(bn / 32) columns, so a chunk
       // may run past bn; columns >= N are never written
@@ -315,15 +363,6 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
                   for (int j = 0; j < 8; ++j)
                     if (col + j < p.N) o[j] = f[j];
                 }
-              } else {  // dX (N is a multiple of 8): bf16(dX + acc)
-                uint16_t* d = p.dx + static_cast<int64_t>(row) * p.dx_ld + col;
-                const uint4 old = *reinterpret_cast<const uint4*>(d);
-                uint4 o;
-                o.x = pack_bf16(bf16lo(old.x) + f[0], bf16hi(old.x) + f[1]);
-                o.y = pack_bf16(bf16lo(old.y) + f[2], bf16hi(old.y) + f[3]);
-                o.z = pack_bf16(bf16lo(old.z) + f[4], bf16hi(old.z) + f[5]);
-                o.w = pack_bf16(bf16lo(old.w) + f[6], bf16hi(old.w) + f[7]);
-                *reinterpret_cast<uint4*>(d) = o;
               }
             }
           }

@@ -43,9 +43,6 @@
 namespace moe {
 
 enum GemmKind : int { kFwdGateUp = 0, kFwdDown = 1, kBwdDgradDown = 2, kBwdDgradGateUp = 3, kBwdWgrad = 4 };
-// Which operand, if any, is read by row gather from a token-order tensor
-// (tmG, rows = token ids sorted_pair[r] / gather_k) instead of a permuted copy.
-enum GatherMode : int { kNoGather = 0, kGatherA = 1, kGatherB = 2 };
 
 constexpr int kBM = 256;        // rows of a pair tile
 constexpr int kBMc = 128;       // rows per CTA
@@ -62,9 +59,14 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 #ifndef MOE_EPI_WARPS
 #define MOE_EPI_WARPS 8
 #endif
+// K blocks the L2 prefetch cursor runs ahead of the TMA loads (0: off).
+#ifndef MOE_PREFETCH_AHEAD
+#define MOE_PREFETCH_AHEAD 0
+#endif
 constexpr int kEpiWarps = MOE_EPI_WARPS;
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "4 or 8 epilogue warps");
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
 // Epilogue outputs are written with the streaming hint (evict-first in L2)
 // so they do not push reused operand tiles out of L2.
 #ifndef MOE_STREAM_STORES
@@ -93,7 +95,6 @@ constexpr int kStageWarpBytes = 32 * kStageStrideBytes;
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
-  CUtensorMap tmG;                 // gathered operand: token-order [gather_rows, K or MN], box 64 x 1
   const CUtensorMap* expert_maps;  // wgrad: [2][E] maps (A then B) clipped at each segment end
   const int32_t* offsets;      // [E+1] expert segment bounds in the permuted rows
   const int32_t* sorted_pair;  // [P]
@@ -113,8 +114,6 @@ struct GemmParams {
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
   float* dw_part;             // BwdDgradDown: [P, kDwSlotsPerNTile * n_tiles] partial routing-weight grads
-  int gather_k;               // pair id -> token: q / gather_k
-  int gather_rows;            // rows of tmG (tokens)
 };
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
@@ -261,10 +260,7 @@ __device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t wro
 __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
-// Warp-uniform read of the CTA's abort flag.
-__device__ __forceinline__ bool warp_aborted(volatile int* s_abort) { return __any_sync(0xffffffffu, *s_abort != 0); }
-
-template <int KIND, int GATHER>
+template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool kWgrad = (KIND == kBwdWgrad);
@@ -315,7 +311,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
-    if constexpr (GATHER != kNoGather) tma_prefetch_desc(&p.tmG);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, kTmemCols);
@@ -356,40 +351,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
-    // Lane 0 waits for a free ring stage, arms the full barrier (even CTA)
-    // and issues the tiled loads. A gathered operand (rows picked by token
-    // index from a token-order tensor instead of a permuted copy) is loaded
-    // by all 32 lanes, one four-row gather per lane per K block.
-    constexpr bool kGather = (GATHER != kNoGather);
-    constexpr bool kGatherMN = kGather && kWgrad;  // gathered rows are K rows (wgrad)
-    const int gk = p.gather_k > 0 ? p.gather_k : 1;
-    // token of pair id q, clamped into the tensor (rows past a segment end
-    // are never used by an output, see below)
-    auto token_of = [&](int32_t q) {
-      const int t = q / gk;
-      return t < 0 ? 0 : (t >= p.gather_rows ? p.gather_rows - 1 : t);
-    };
-    // Row-grouped kinds: lane l gathers rows 4l..4l+3 of this CTA's 128 tile
-    // rows for every K block of the tile; rows past the segment end load
-    // token 0 and their outputs are masked by the epilogue.
-    auto tile_pairs = [&](const TileInfo& ti, int32_t (&q)[4]) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int r = static_cast<int>(rank) * kBMc + 4 * lane + m;
-        q[m] = r < ti.rows ? __ldg(p.sorted_pair + ti.row0 + r) : 0;
-      }
-    };
-    // Wgrad: K block kb covers the segment's rows 64kb..64kb+63; lane l
-    // gathers rows 4(l%16)..+3 into MN chunk l/16. Rows past the segment
-    // end load token 0; the other operand's per-expert map reads zeros there.
-    auto kblock_pairs = [&](const TileInfo& ti, int kb, int32_t (&q)[4]) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int r = kb * kBK + 4 * (lane & 15) + m;
-        q[m] = (kb < ti.num_kb && r < ti.rows) ? __ldg(p.sorted_pair + ti.row0 + r) : 0;
-      }
-    };
-    auto issue = [&](const TileInfo& ti, int kb, uint8_t* a_dst, uint8_t* b_dst, uint32_t fb, const int32_t (&q)[4]) {
+    // Loads K block kb of tile ti (this CTA's A half and B half) into a ring
+    // stage, or with prefetch_only just asks TMA to bring the same boxes into
+    // L2. A prefetch cursor runs kPrefetchAhead K blocks (across tile
+    // boundaries) ahead of the loads so first touches of weight and
+    // activation tiles start their DRAM reads early.
+    auto issue = [&](const TileInfo& ti, int kb, bool prefetch_only, uint8_t* a_dst, uint8_t* b_dst, uint32_t fb) {
       const CUtensorMap* mapA = &p.tmA;
       const CUtensorMap* mapB = &p.tmB;
       if constexpr (kWgrad) {
@@ -415,88 +382,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         nbox_a = 2;
         nbox_b = 2;
       }
-      if (lane == 0) {
-        if constexpr (GATHER != kGatherA)
-          for (int c = 0; c < nbox_a; ++c) tma_load_2d_pair(a_dst + 8192 * c, mapA, fb, ax + 64 * c, ay);
-        if constexpr (GATHER != kGatherB)
-          for (int c = 0; c < nbox_b; ++c) tma_load_2d_pair(b_dst + 8192 * c, mapB, fb, bx + 64 * c, by);
+      for (int c = 0; c < nbox_a; ++c) {
+        if (prefetch_only) tma_prefetch_2d(mapA, ax + 64 * c, ay);
+        else tma_load_2d_pair(a_dst + 8192 * c, mapA, fb, ax + 64 * c, ay);
       }
-      if constexpr (kGather) {
-        uint8_t* g_dst = (GATHER == kGatherA) ? a_dst : b_dst;
-        int gx = kx, goff = 512 * lane;
-        if constexpr (kGatherMN) {
-          const int chunk = lane >> 4;
-          gx = ((GATHER == kGatherA) ? ax : bx) + 64 * chunk;
-          goff = 8192 * chunk + 512 * (lane & 15);
-        }
-        tma_gather4_pair(g_dst + goff, &p.tmG, fb, gx, token_of(q[0]), token_of(q[1]), token_of(q[2]),
-                         token_of(q[3]));
+      for (int c = 0; c < nbox_b; ++c) {
+        if (prefetch_only) tma_prefetch_2d(mapB, bx + 64 * c, by);
+        else tma_load_2d_pair(b_dst + 8192 * c, mapB, fb, bx + 64 * c, by);
       }
     };
-    int stage = 0;
-    uint32_t phase = 0;
-    int issued = 0;
-    int32_t q_cur[4] = {0, 0, 0, 0}, q_nxt[4] = {0, 0, 0, 0};
-    if constexpr (kGather && !kGatherMN) {
-      if (pair < total_tiles) tile_pairs(decode_tile<KIND>(pair, p, s_off, s_tstart), q_nxt);
-    }
-    for (int t = pair; t < total_tiles && !warp_aborted(s_abort); t += num_pairs) {
-      const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
-      if constexpr (kWgrad) {
-        if (ti.num_kb == 0) continue;
-        if (lane == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      // prefetch cursor: tile pf_t, K block pf_kb; pf_lead = blocks ahead of the loads
+      int pf_t = pair, pf_kb = 0, pf_lead = 0;
+      TileInfo pf_ti;
+      if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
+      for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
+        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        if constexpr (kWgrad) {
+          if (ti.num_kb == 0) continue;
           tensormap_acquire(p.expert_maps + ti.e);
           tensormap_acquire(p.expert_maps + p.E + ti.e);
         }
-      }
-      // gathered pair ids: the tile's (row-grouped, requested one tile
-      // ahead) or the next K blocks' (wgrad, requested two blocks ahead)
-      int32_t q_k1[4] = {0, 0, 0, 0}, q_k2[4] = {0, 0, 0, 0};
-      if constexpr (kGather && !kGatherMN) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) q_cur[m] = q_nxt[m];
-        if (t + num_pairs < total_tiles) tile_pairs(decode_tile<KIND>(t + num_pairs, p, s_off, s_tstart), q_nxt);
-      }
-      if constexpr (kGatherMN) {
-        kblock_pairs(ti, 0, q_k1);
-        kblock_pairs(ti, 1, q_k2);
-      }
-      for (int kb = 0; kb < ti.num_kb; ++kb) {
-        if constexpr (kGatherMN) {
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            q_cur[m] = q_k1[m];
-            q_k1[m] = q_k2[m];
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          while (pf_lead < kPrefetchAhead && pf_t < total_tiles) {
+            if (pf_kb < pf_ti.num_kb) {
+              if constexpr (kWgrad) {
+                if (pf_kb == 0) {
+                  tensormap_acquire(p.expert_maps + pf_ti.e);
+                  tensormap_acquire(p.expert_maps + p.E + pf_ti.e);
+                }
+              }
+              issue(pf_ti, pf_kb, true, nullptr, nullptr, 0);
+              ++pf_kb;
+              ++pf_lead;
+            } else {
+              pf_t += num_pairs;
+              pf_kb = 0;
+              if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
+            }
           }
-          kblock_pairs(ti, kb + 2, q_k2);
-        }
-        if (!warp_wait(&empty_bar[stage], phase ^ 1u)) {
-          if (lane == 0) report(MOE_ERR_TIMEOUT);
-          *s_abort = 1;
-          break;
-        }
-        if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
-        __syncwarp();
-        issue(ti, kb, sA + stage * kATileBytes, sB + stage * kBTileBytes,
-              mapa_shared(smem_u32(&full_bar[stage]), 0), q_cur);
-        ++issued;
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+            report(MOE_ERR_TIMEOUT);
+            *s_abort = 1;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
+          issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes,
+                mapa_shared(smem_u32(&full_bar[stage]), 0));
+          if (pf_lead > 0) --pf_lead;
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
-    }
-    // The even CTA's full barriers count both CTAs' bytes: waiting on the
-    // last phases there means no load of the pair is still in flight when
-    // the pair leaves (immediate in normal operation).
-    if (lane == 0 && rank == 0) {
-      const int inflight = issued < kStages ? issued : kStages;
-      for (int i = 0; i < inflight; ++i) {
-        if (--stage < 0) {
-          stage = kStages - 1;
-          phase ^= 1u;
+      // The even CTA's full barriers count both CTAs' bytes: waiting on the
+      // last phases there means no load of the pair is still in flight when
+      // the pair leaves (immediate in normal operation).
+      if (rank == 0) {
+        const int inflight = issued < kStages ? issued : kStages;
+        for (int i = 0; i < inflight; ++i) {
+          if (--stage < 0) {
+            stage = kStages - 1;
+            phase ^= 1u;
+          }
+          mbar_wait(&full_bar[stage], phase);
         }
-        mbar_wait(&full_bar[stage], phase);
       }
     }
   } else if (warp == 1) {
@@ -507,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int tcount = 0;
-      for (int t = pair; t < total_tiles && !warp_aborted(s_abort); t += num_pairs) {
+      for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
         const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
         if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogues write zeros
         const int acc = tcount & 1;
@@ -577,7 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
     constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / (kEpiWarps / 4);  // chunks per warp
     int tcount = 0;
-    for (int t = pair; t < total_tiles && !warp_aborted(s_abort); t += num_pairs) {
+    for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
       const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
       // this CTA's 128 rows of the pair tile, this warp's 32 of them
       const int cta_row0 = static_cast<int>(rank) * kBMc + sub * 32;

@@ -115,12 +115,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-gather map of a token-order bf16 tensor [rows, inner]: 64-column boxes
-// one row high (the tile::gather4 form).
-bool make_gather_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
-  return make_map(m, base, inner, rows, 64, 1);
-}
-
 // ---------------------------------------------------------------- profiling
 enum ProfSlot : int {
   kProfRoute = 0,
@@ -203,14 +197,14 @@ struct ProfScope {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-template <int KIND, int GATHER = kNoGather>
+template <int KIND>
 int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
   const size_t smem = gemm_smem_bytes(p.E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
   ProfScope ps(slot, s);
-  if (launch_pdl(grouped_gemm_kernel<KIND, GATHER>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
+  if (launch_pdl(grouped_gemm_kernel<KIND>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_status();
 }
@@ -245,12 +239,11 @@ bool dims_ok(int H) { return H > 0 && H % 8 == 0; }
 struct BwdLayout {
   size_t dYp, dGU, hw, dXp, dw_part, maps, gu, total;
 };
-// gather: the backward reads dY and X by row gather (no dYp copy).
-BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute, bool gather = false) {
+BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
   const size_t P = static_cast<size_t>(T) * k;
   BwdLayout L;
   size_t off = 0;
-  L.dYp = off; off += gather ? 0 : round256(P * H * 2);
+  L.dYp = off; off += round256(P * H * 2);
   L.dGU = off; off += round256(P * 2 * I * 2);
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
@@ -486,16 +479,9 @@ int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* c
                      sizeof(int) * static_cast<size_t>(kNoAllocPermuteScratchInts), stream);
 }
 
-}  // extern "C"
-
-namespace moe {
-namespace {
-// The two expert GEMMs of the forward. gather: `src` is X [T, H] in token
-// order and the gate/up GEMM gathers its rows; otherwise `src` is Xp [P, H].
-int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, const int32_t* sorted_pair,
-                     const float* topk_w, int T, int E, int k, int H, int I, const moe_bf16* W_gu,
-                     const moe_bf16* W_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, cudaStream_t stream) {
-  const moe_bf16* Xp = src;
+int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
   if (P == 0) return MOE_OK;
@@ -506,15 +492,8 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   if (int st = current_device_info(&dev)) return st;
 
   GemmParams gu = base_params(E, P, offsets);
-  if (gather) {
-    if (!make_gather_map(&gu.tmG, src, H, T)) return MOE_ERR_CUDA;
-    gu.tmA = gu.tmG;  // not loaded from; keeps the descriptor prefetch on a valid map
-    gu.gather_k = k;
-    gu.gather_rows = T;
-  } else if (!make_map(&gu.tmA, Xp, H, P, 64, 128)) {
+  if (!make_map(&gu.tmA, Xp, H, P, 64, 128) || !make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
     return MOE_ERR_CUDA;
-  }
-  if (!make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
   gu.sorted_pair = sorted_pair;
   gu.N = I;
   gu.K = H;
@@ -524,9 +503,7 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   gu.out = h;
   gu.out_ld = I;
   gu.gu = gu_save;
-  const int gu_grid = rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms);
-  if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(gu, gu_grid, stream, kProfFwdGateUp)
-                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp))
+  if (int st = launch_gemm<kFwdGateUp>(gu, rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms), stream, kProfFwdGateUp))
     return st;
 
   GemmParams dn = base_params(E, P, offsets);
@@ -542,22 +519,6 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   dn.out = O;
   dn.out_ld = H;
   return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown);
-}
-}  // namespace
-}  // namespace moe
-
-extern "C" {
-
-int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
-                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
-                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
-  return experts_fwd_impl(Xp, false, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, h, gu_save, O, stream);
-}
-
-int moe_experts_fwd_x(const moe_bf16* X, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
-                      int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
-                      moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
-  return experts_fwd_impl(X, true, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, h, gu_save, O, stream);
 }
 
 int moe_combine(const moe_bf16* O, const int32_t* pair_pos, int T, int k, int H, moe_bf16* Y, moe_stream_t stream) {
@@ -575,24 +536,11 @@ size_t moe_layer_bwd_workspace_bytes(int T, int E, int k, int H, int I, int reco
   return bwd_layout(T, E, k, H, I, recompute_gu != 0).total;
 }
 
-size_t moe_layer_bwd_x_workspace_bytes(int T, int E, int k, int H, int I, int recompute_gu) {
-  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return 0;
-  return bwd_layout(T, E, k, H, I, recompute_gu != 0, true).total;
-}
-
-}  // extern "C"
-
-namespace moe {
-namespace {
-// The layer's backward. gather: `src` is X [T, H] in token order and the
-// GEMMs that read X or dY rows gather them (no dYp copy, no gather kernel);
-// otherwise `src` is Xp [P, H] and dY is first gathered into dYp.
-int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const moe_bf16* gu_save,
-                   const moe_bf16* h, const float* probs, const int32_t* topk_idx, const float* topk_w,
-                   const int32_t* offsets, const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k,
-                   int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu,
-                   moe_bf16* dW_d, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  const moe_bf16* Xp = src;
+int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
@@ -602,7 +550,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     return MOE_ERR_INVALID_ARG;
   (void)h;  // not read: the dgrad-down epilogue recomputes h = silu(g) * u from g|u
   const bool recompute = (gu_save == nullptr);
-  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute, gather);
+  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute);
   if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
@@ -622,8 +570,8 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   float* dw_part = reinterpret_cast<float*>(w8 + L.dw_part);
   const int nt_dgrad_down = cdiv(I, kBN);
 
-  // 1. dYp[r] = dY[token of row r] (gathered by the GEMMs instead when gather)
-  if (!gather) {
+  // 1. dYp[r] = dY[token of row r]
+  {
     ProfScope ps(kProfGatherDy, stream);
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
@@ -637,15 +585,9 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   if (recompute) {
     moe_bf16* gu_ws = reinterpret_cast<moe_bf16*>(w8 + L.gu);
     GemmParams rc = base_params(E, P, offsets);
-    if (gather) {
-      if (!make_gather_map(&rc.tmG, src, H, T)) return MOE_ERR_CUDA;
-      rc.tmA = rc.tmG;
-      rc.gather_k = k;
-      rc.gather_rows = T;
-    } else if (!make_map(&rc.tmA, Xp, H, P, 64, 128)) {
+    if (!make_map(&rc.tmA, Xp, H, P, 64, 128) ||
+        !make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
       return MOE_ERR_CUDA;
-    }
-    if (!make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
     rc.sorted_pair = sorted_pair;
     rc.N = I;
     rc.K = H;
@@ -654,24 +596,17 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     rc.n_tiles = cdiv(I, 128);
     rc.out = nullptr;
     rc.gu = gu_ws;
-    const int grid = rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms);
-    if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(rc, grid, stream, kProfRecomputeGateUp)
-                        : launch_gemm<kFwdGateUp>(rc, grid, stream, kProfRecomputeGateUp))
+    if (int st = launch_gemm<kFwdGateUp>(rc, rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms), stream,
+                                         kProfRecomputeGateUp))
       return st;
     gu = gu_ws;
   }
   // 3. dgrad through down + SwiGLU backward: dGU, hw, partial dw
   {
     GemmParams bd = base_params(E, P, offsets);
-    if (gather) {
-      if (!make_gather_map(&bd.tmG, dY, H, T)) return MOE_ERR_CUDA;
-      bd.tmA = bd.tmG;
-      bd.gather_k = k;
-      bd.gather_rows = T;
-    } else if (!make_map(&bd.tmA, dYp, H, P, 64, 128)) {
+    if (!make_map(&bd.tmA, dYp, H, P, 64, 128) ||
+        !make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64))
       return MOE_ERR_CUDA;
-    }
-    if (!make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64)) return MOE_ERR_CUDA;
     bd.sorted_pair = sorted_pair;
     bd.topk_w = topk_w;
     bd.N = I;
@@ -684,9 +619,8 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     bd.gu = const_cast<moe_bf16*>(gu);
     bd.hw_out = hw;
     bd.dw_part = dw_part;
-    const int grid = rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms);
-    if (int st = gather ? launch_gemm<kBwdDgradDown, kGatherA>(bd, grid, stream, kProfDgradDown)
-                        : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown))
+    if (int st = launch_gemm<kBwdDgradDown>(bd, rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms), stream,
+                                            kProfDgradDown))
       return st;
   }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
@@ -716,15 +650,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(w8 + L.maps);
   {
     GemmParams wg = base_params(E, P, offsets);
-    if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64)) return MOE_ERR_CUDA;
-    if (gather) {  // B = X rows gathered by token (its per-expert map copy is unused)
-      if (!make_gather_map(&wg.tmG, src, H, T)) return MOE_ERR_CUDA;
-      wg.tmB = wg.tmG;
-      wg.gather_k = k;
-      wg.gather_rows = T;
-    } else if (!make_map(&wg.tmB, Xp, H, P, 64, 64)) {
-      return MOE_ERR_CUDA;
-    }
+    if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64) || !make_map(&wg.tmB, Xp, H, P, 64, 64)) return MOE_ERR_CUDA;
     if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wg.tmA, wg.tmB, offsets, E,
                    maps) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -738,22 +664,11 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wg.out_ld = H;
     wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
     const int64_t tiles = static_cast<int64_t>(E) * wg.m_tiles * wg.n_tiles;
-    const int grid = pair_grid(tiles, dev->num_sms);
-    if (int st = gather ? launch_gemm<kBwdWgrad, kGatherB>(wg, grid, stream, kProfWgradGateUp)
-                        : launch_gemm<kBwdWgrad>(wg, grid, stream, kProfWgradGateUp))
-      return st;
+    if (int st = launch_gemm<kBwdWgrad>(wg, pair_grid(tiles, dev->num_sms), stream, kProfWgradGateUp)) return st;
   }
   {
     GemmParams wd = base_params(E, P, offsets);
-    if (gather) {  // A = dY rows gathered by token (its per-expert map copy is unused)
-      if (!make_gather_map(&wd.tmG, dY, H, T)) return MOE_ERR_CUDA;
-      wd.tmA = wd.tmG;
-      wd.gather_k = k;
-      wd.gather_rows = T;
-    } else if (!make_map(&wd.tmA, dYp, H, P, 64, 64)) {
-      return MOE_ERR_CUDA;
-    }
-    if (!make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
+    if (!make_map(&wd.tmA, dYp, H, P, 64, 64) || !make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
     if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wd.tmA, wd.tmB, offsets, E,
                    maps + 2 * E) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -767,10 +682,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wd.out_ld = I;
     wd.out_expert_stride = static_cast<int64_t>(H) * I;
     const int64_t tiles = static_cast<int64_t>(E) * wd.m_tiles * wd.n_tiles;
-    const int grid = pair_grid(tiles, dev->num_sms);
-    if (int st = gather ? launch_gemm<kBwdWgrad, kGatherA>(wd, grid, stream, kProfWgradDown)
-                        : launch_gemm<kBwdWgrad>(wd, grid, stream, kProfWgradDown))
-      return st;
+    if (int st = launch_gemm<kBwdWgrad>(wd, pair_grid(tiles, dev->num_sms), stream, kProfWgradDown)) return st;
   }
   // 7. router logits gradient
   {
@@ -783,28 +695,6 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
       return MOE_ERR_CUDA;
   }
   return MOE_OK;
-}
-}  // namespace
-}  // namespace moe
-
-extern "C" {
-
-int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
-                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
-                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
-                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
-                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
-                        H, I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
-}
-
-int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
-                    const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
-                    const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
-                    const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
-                    float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  return layer_bwd_impl(dY, X, true, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k, H,
-                        I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
 }
 
 size_t moe_router_workspace_bytes(int T, int H, int E) {

@@ -221,21 +221,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
-// Row-gather TMA load into this CTA's shared memory: four rows (row0..row3)
-// of a 2-D tensor whose map has a box one row high, columns x..x+box-1,
-// written as four consecutive box rows (same swizzle as a tiled load at that
-// address); completion bytes are counted on an mbarrier of either CTA of the
-// pair (cluster address).
-__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
-                                                 int x, int row0, int row1, int row2, int row3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(row0), "r"(row1), "r"(row2),
-      "r"(row3)
-      : "memory");
-}
-
 // --------------------------------------------------- tcgen05 for CTA pairs
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),

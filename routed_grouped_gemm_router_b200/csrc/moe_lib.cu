@@ -197,29 +197,16 @@ struct ProfScope {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-template <int KIND, int CG>
-int launch_gemm_instance(const GemmParams& p, int grid, cudaStream_t s) {
-  const size_t smem = gemm_smem_bytes<CG>(p.E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int KIND>
+int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
+  const size_t smem = gemm_smem_bytes(p.E);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_pdl_clustered(grouped_gemm_kernel<KIND, CG>, dim3(grid), dim3(kGemmThreads), smem, s,
-                           static_cast<unsigned>(CG), p) != cudaSuccess)
+  ProfScope ps(slot, s);
+  if (launch_pdl(grouped_gemm_kernel<KIND>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_status();
-}
-
-// One grouped GEMM: the pair instance over its tiles (grid = CTA pairs), then
-// for the row-grouped kinds the one-CTA instance over the segment tails of
-// 1..128 rows (tail_grid CTAs).
-template <int KIND>
-int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot, int tail_grid = 0) {
-  ProfScope ps(slot, s);
-  if (int st = launch_gemm_instance<KIND, 2>(p, grid, s)) return st;
-  if constexpr (KIND != kBwdWgrad) {
-    if (kTailTiles && tail_grid > 0) return launch_gemm_instance<KIND, 1>(p, tail_grid, s);
-  }
-  return MOE_OK;
 }
 
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -233,11 +220,6 @@ inline int pair_grid(int64_t tiles, int num_sms) {
 }
 inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
   return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
-}
-// One-CTA instance: at most one tail tile per expert and N block, one CTA per SM.
-inline int tail_grid(int E, int n_tiles, int num_sms) {
-  const int64_t tiles = static_cast<int64_t>(E) * n_tiles;
-  return static_cast<int>(tiles < num_sms ? tiles : num_sms);
 }
 
 GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
@@ -521,7 +503,7 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   gu.out = h;
   gu.out_ld = I;
   gu.gu = gu_save;
-  if (int st = launch_gemm<kFwdGateUp>(gu, rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms), stream, kProfFwdGateUp, tail_grid(E, gu.n_tiles, dev->num_sms)))
+  if (int st = launch_gemm<kFwdGateUp>(gu, rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms), stream, kProfFwdGateUp))
     return st;
 
   GemmParams dn = base_params(E, P, offsets);
@@ -536,7 +518,7 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   dn.n_tiles = cdiv(H, kBN);
   dn.out = O;
   dn.out_ld = H;
-  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown, tail_grid(E, dn.n_tiles, dev->num_sms));
+  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown);
 }
 
 int moe_combine(const moe_bf16* O, const int32_t* pair_pos, int T, int k, int H, moe_bf16* Y, moe_stream_t stream) {
@@ -615,7 +597,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     rc.out = nullptr;
     rc.gu = gu_ws;
     if (int st = launch_gemm<kFwdGateUp>(rc, rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms), stream,
-                                         kProfRecomputeGateUp, tail_grid(E, rc.n_tiles, dev->num_sms)))
+                                         kProfRecomputeGateUp))
       return st;
     gu = gu_ws;
   }
@@ -638,7 +620,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     bd.hw_out = hw;
     bd.dw_part = dw_part;
     if (int st = launch_gemm<kBwdDgradDown>(bd, rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms), stream,
-                                            kProfDgradDown, tail_grid(E, bd.n_tiles, dev->num_sms)))
+                                            kProfDgradDown))
       return st;
   }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
@@ -655,7 +637,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     bx.out = dXp;
     bx.out_ld = H;
     if (int st = launch_gemm<kBwdDgradGateUp>(bx, rowgrouped_grid(P, E, bx.n_tiles, dev->num_sms), stream,
-                                              kProfDgradGateUp, tail_grid(E, bx.n_tiles, dev->num_sms)))
+                                              kProfDgradGateUp))
       return st;
   }
   // 5. dX[t] = sum_j dXp[pair_pos[t*k+j]]

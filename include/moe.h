@@ -202,6 +202,32 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Gather-fused variants -- the same results as moe_experts_fwd and
+ * moe_layer_bwd, reading the activations in token order: the GEMMs load the
+ * rows of X [T,H] (and of dY [T,H]) by token index t = sorted_pair[r] / k
+ * with 16-byte asynchronous copies issued by the GEMM itself, so no permuted
+ * copies Xp / dYp are made or read.
+ * Source: fused-MoE Triton project summary (sourcepulse), How It Works:
+ * inputs are sorted by expert for coalesced grouped-GEMM reads; here the
+ * sort is applied inside the GEMM's operand loads. moe_permute may then be
+ * called with X = Xp = NULL.
+ */
+int moe_experts_fwd_x(const moe_bf16* X, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                      int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                      moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream);
+
+/* Scratch bytes of moe_layer_bwd_x (smaller than moe_layer_bwd's: no dYp). */
+size_t moe_layer_bwd_x_workspace_bytes(int T, int E, int k, int H, int I, int recompute_gu);
+
+/* moe_layer_bwd with X [T,H] in token order in place of Xp;
+ * ws >= moe_layer_bwd_x_workspace_bytes(...). */
+int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
+                    const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                    const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                    const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                    float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Router Linear -- logits = X W_r^T and its backward, on the tensor cores.
  * Source: "Integration of fused moe kernel (e.g., megablocks) for efficient
  * moe training" (axolotl issue #3155), discussion of the router's weight

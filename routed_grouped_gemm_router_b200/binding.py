@@ -32,9 +32,13 @@ _SIGNATURES = {
                                      _c_void, _c_int, _c_void, _c_void]),
     "moe_experts_fwd": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
                                  _c_void, _c_void, _c_void, _c_void, _c_void, _c_void]),
+    "moe_experts_fwd_x": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _c_void, _c_void, _c_void, _c_void, _c_void, _c_void]),
     "moe_combine": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_void, _c_void]),
     "moe_layer_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
+    "moe_layer_bwd_x_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "moe_layer_bwd_x": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
     "moe_router_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_router_fwd": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void,
                                 _c_void, _c_void, _c_size, _c_void]),
@@ -150,19 +154,21 @@ def moe_permute(topk_idx: torch.Tensor, E: int, X: torch.Tensor | None = None, o
 
 
 def moe_experts_fwd(Xp, offsets, sorted_pair, topk_w, T, E, k, W_gu, W_d, h=None, gu_save=None, O=None,
-                    save_gu=True, stream=None):
+                    save_gu=True, stream=None, gather=False):
+    """gather=True: `Xp` is X [T, H] in token order (moe_experts_fwd_x)."""
     P = T * k
     H = W_gu.shape[2]
     I = W_d.shape[2]
     dev = Xp.device
-    _need(Xp, torch.bfloat16, (P, H), "Xp")
+    _need(Xp, torch.bfloat16, (T if gather else P, H), "X" if gather else "Xp")
     _need(W_gu, torch.bfloat16, (E, 2 * I, H), "W_gu")
     _need(W_d, torch.bfloat16, (E, H, I), "W_d")
     h = torch.empty(P, I, dtype=torch.bfloat16, device=dev) if h is None else h
     if gu_save is None and save_gu:
         gu_save = torch.empty(P, 2 * I, dtype=torch.bfloat16, device=dev)
     O = torch.empty(P, H, dtype=torch.bfloat16, device=dev) if O is None else O
-    _check("moe_experts_fwd", lib().moe_experts_fwd(
+    name = "moe_experts_fwd_x" if gather else "moe_experts_fwd"
+    _check(name, getattr(lib(), name)(
         _ptr(Xp), _ptr(offsets), _ptr(sorted_pair), _ptr(topk_w), T, E, k, H, I, _ptr(W_gu), _ptr(W_d),
         _ptr(h), _ptr(gu_save), _ptr(O), _stream(stream)))
     return h, gu_save, O
@@ -176,7 +182,8 @@ def moe_combine(O, pair_pos, T, k, Y=None, stream=None):
 
 
 def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
-                  W_gu, W_d, out=None, ws=None, stream=None):
+                  W_gu, W_d, out=None, ws=None, stream=None, gather=False):
+    """gather=True: `Xp` is X [T, H] in token order (moe_layer_bwd_x)."""
     H = W_gu.shape[2]
     I = W_d.shape[2]
     dev = dY.device
@@ -185,10 +192,12 @@ def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_p
     o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev))
     o.setdefault("dW_d", torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
     o.setdefault("dlogits", torch.empty(T, E, dtype=torch.float32, device=dev))
-    need = lib().moe_layer_bwd_workspace_bytes(T, E, k, H, I, 1 if gu_save is None else 0)
+    query = lib().moe_layer_bwd_x_workspace_bytes if gather else lib().moe_layer_bwd_workspace_bytes
+    need = query(T, E, k, H, I, 1 if gu_save is None else 0)
     if ws is None:
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    _check("moe_layer_bwd", lib().moe_layer_bwd(
+    name = "moe_layer_bwd_x" if gather else "moe_layer_bwd"
+    _check(name, getattr(lib(), name)(
         _ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
         _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]),
         _ptr(o["dW_gu"]), _ptr(o["dW_d"]), _ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream)))

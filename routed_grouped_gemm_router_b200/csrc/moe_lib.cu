@@ -197,14 +197,14 @@ struct ProfScope {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-template <int KIND>
+template <int KIND, int GATHER = kNoGather>
 int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
   const size_t smem = gemm_smem_bytes(p.E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
   ProfScope ps(slot, s);
-  if (launch_pdl(grouped_gemm_kernel<KIND>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
+  if (launch_pdl(grouped_gemm_kernel<KIND, GATHER>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_status();
 }
@@ -220,6 +220,16 @@ inline int pair_grid(int64_t tiles, int num_sms) {
 }
 inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
   return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
+}
+
+// The gathered operand of a GEMM: token-order rows [T, H] picked by
+// sorted_pair[r] / k. Its tensor map is not loaded from; a valid map is kept
+// in its place for the kernel's descriptor prefetch.
+void set_gather(GemmParams& g, const moe_bf16* src, int T, int k, int H) {
+  g.gsrc = src;
+  g.gather_k = k;
+  g.gather_rows = T;
+  g.gather_cols = H;
 }
 
 GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
@@ -239,11 +249,12 @@ bool dims_ok(int H) { return H > 0 && H % 8 == 0; }
 struct BwdLayout {
   size_t dYp, dGU, hw, dXp, dw_part, maps, gu, total;
 };
-BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute) {
+// gather: the GEMMs read dY (and X) rows by token, so there is no dYp copy.
+BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute, bool gather = false) {
   const size_t P = static_cast<size_t>(T) * k;
   BwdLayout L;
   size_t off = 0;
-  L.dYp = off; off += round256(P * H * 2);
+  L.dYp = off; off += gather ? 0 : round256(P * H * 2);
   L.dGU = off; off += round256(P * 2 * I * 2);
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
@@ -479,9 +490,16 @@ int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* c
                      sizeof(int) * static_cast<size_t>(kNoAllocPermuteScratchInts), stream);
 }
 
-int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
-                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
-                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+// The two expert GEMMs of the forward. gather: `src` is X [T, H] in token
+// order and the gate/up GEMM gathers its rows; otherwise `src` is Xp [P, H].
+int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, const int32_t* sorted_pair,
+                     const float* topk_w, int T, int E, int k, int H, int I, const moe_bf16* W_gu,
+                     const moe_bf16* W_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, cudaStream_t stream) {
+  const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
   if (P == 0) return MOE_OK;
@@ -492,8 +510,13 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   if (int st = current_device_info(&dev)) return st;
 
   GemmParams gu = base_params(E, P, offsets);
-  if (!make_map(&gu.tmA, Xp, H, P, 64, 128) || !make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
+  if (!make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
+  if (gather) {
+    set_gather(gu, src, T, k, H);
+    gu.tmA = gu.tmB;
+  } else if (!make_map(&gu.tmA, Xp, H, P, 64, 128)) {
     return MOE_ERR_CUDA;
+  }
   gu.sorted_pair = sorted_pair;
   gu.N = I;
   gu.K = H;
@@ -503,7 +526,9 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   gu.out = h;
   gu.out_ld = I;
   gu.gu = gu_save;
-  if (int st = launch_gemm<kFwdGateUp>(gu, rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms), stream, kProfFwdGateUp))
+  const int gu_grid = rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms);
+  if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(gu, gu_grid, stream, kProfFwdGateUp)
+                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp))
     return st;
 
   GemmParams dn = base_params(E, P, offsets);
@@ -519,6 +544,22 @@ int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* s
   dn.out = O;
   dn.out_ld = H;
   return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown);
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_experts_fwd(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                    int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                    moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
+  return experts_fwd_impl(Xp, false, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, h, gu_save, O, stream);
+}
+
+int moe_experts_fwd_x(const moe_bf16* X, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                      int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* h,
+                      moe_bf16* gu_save, moe_bf16* O, moe_stream_t stream) {
+  return experts_fwd_impl(X, true, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, h, gu_save, O, stream);
 }
 
 int moe_combine(const moe_bf16* O, const int32_t* pair_pos, int T, int k, int H, moe_bf16* Y, moe_stream_t stream) {
@@ -536,11 +577,24 @@ size_t moe_layer_bwd_workspace_bytes(int T, int E, int k, int H, int I, int reco
   return bwd_layout(T, E, k, H, I, recompute_gu != 0).total;
 }
 
-int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
-                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
-                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
-                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
-                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+size_t moe_layer_bwd_x_workspace_bytes(int T, int E, int k, int H, int I, int recompute_gu) {
+  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return 0;
+  return bwd_layout(T, E, k, H, I, recompute_gu != 0, true).total;
+}
+
+}  // extern "C"
+
+namespace moe {
+namespace {
+// The layer's backward. gather: `src` is X [T, H] in token order and the
+// GEMMs that read X or dY rows gather them (no dYp copy, no gather kernel);
+// otherwise `src` is Xp [P, H] and dY is first gathered into dYp.
+int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const moe_bf16* gu_save,
+                   const moe_bf16* h, const float* probs, const int32_t* topk_idx, const float* topk_w,
+                   const int32_t* offsets, const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k,
+                   int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu,
+                   moe_bf16* dW_d, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
@@ -550,7 +604,7 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     return MOE_ERR_INVALID_ARG;
   (void)h;  // not read: the dgrad-down epilogue recomputes h = silu(g) * u from g|u
   const bool recompute = (gu_save == nullptr);
-  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute);
+  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute, gather);
   if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
@@ -570,8 +624,8 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   float* dw_part = reinterpret_cast<float*>(w8 + L.dw_part);
   const int nt_dgrad_down = cdiv(I, kBN);
 
-  // 1. dYp[r] = dY[token of row r]
-  {
+  // 1. dYp[r] = dY[token of row r] (the GEMMs gather dY themselves when gather)
+  if (!gather) {
     ProfScope ps(kProfGatherDy, stream);
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
@@ -585,9 +639,13 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   if (recompute) {
     moe_bf16* gu_ws = reinterpret_cast<moe_bf16*>(w8 + L.gu);
     GemmParams rc = base_params(E, P, offsets);
-    if (!make_map(&rc.tmA, Xp, H, P, 64, 128) ||
-        !make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128))
+    if (!make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
+    if (gather) {
+      set_gather(rc, src, T, k, H);
+      rc.tmA = rc.tmB;
+    } else if (!make_map(&rc.tmA, Xp, H, P, 64, 128)) {
       return MOE_ERR_CUDA;
+    }
     rc.sorted_pair = sorted_pair;
     rc.N = I;
     rc.K = H;
@@ -596,17 +654,22 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     rc.n_tiles = cdiv(I, 128);
     rc.out = nullptr;
     rc.gu = gu_ws;
-    if (int st = launch_gemm<kFwdGateUp>(rc, rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms), stream,
-                                         kProfRecomputeGateUp))
+    const int grid = rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms);
+    if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(rc, grid, stream, kProfRecomputeGateUp)
+                        : launch_gemm<kFwdGateUp>(rc, grid, stream, kProfRecomputeGateUp))
       return st;
     gu = gu_ws;
   }
   // 3. dgrad through down + SwiGLU backward: dGU, hw, partial dw
   {
     GemmParams bd = base_params(E, P, offsets);
-    if (!make_map(&bd.tmA, dYp, H, P, 64, 128) ||
-        !make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64))
+    if (!make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64)) return MOE_ERR_CUDA;
+    if (gather) {
+      set_gather(bd, dY, T, k, H);
+      bd.tmA = bd.tmB;
+    } else if (!make_map(&bd.tmA, dYp, H, P, 64, 128)) {
       return MOE_ERR_CUDA;
+    }
     bd.sorted_pair = sorted_pair;
     bd.topk_w = topk_w;
     bd.N = I;
@@ -619,8 +682,9 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     bd.gu = const_cast<moe_bf16*>(gu);
     bd.hw_out = hw;
     bd.dw_part = dw_part;
-    if (int st = launch_gemm<kBwdDgradDown>(bd, rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms), stream,
-                                            kProfDgradDown))
+    const int grid = rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms);
+    if (int st = gather ? launch_gemm<kBwdDgradDown, kGatherA>(bd, grid, stream, kProfDgradDown)
+                        : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown))
       return st;
   }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
@@ -650,7 +714,13 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(w8 + L.maps);
   {
     GemmParams wg = base_params(E, P, offsets);
-    if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64) || !make_map(&wg.tmB, Xp, H, P, 64, 64)) return MOE_ERR_CUDA;
+    if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64)) return MOE_ERR_CUDA;
+    if (gather) {  // B = X rows by token (its per-expert map copy is unused)
+      set_gather(wg, src, T, k, H);
+      wg.tmB = wg.tmA;
+    } else if (!make_map(&wg.tmB, Xp, H, P, 64, 64)) {
+      return MOE_ERR_CUDA;
+    }
     if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wg.tmA, wg.tmB, offsets, E,
                    maps) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -664,11 +734,20 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     wg.out_ld = H;
     wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
     const int64_t tiles = static_cast<int64_t>(E) * wg.m_tiles * wg.n_tiles;
-    if (int st = launch_gemm<kBwdWgrad>(wg, pair_grid(tiles, dev->num_sms), stream, kProfWgradGateUp)) return st;
+    const int grid = pair_grid(tiles, dev->num_sms);
+    if (int st = gather ? launch_gemm<kBwdWgrad, kGatherB>(wg, grid, stream, kProfWgradGateUp)
+                        : launch_gemm<kBwdWgrad>(wg, grid, stream, kProfWgradGateUp))
+      return st;
   }
   {
     GemmParams wd = base_params(E, P, offsets);
-    if (!make_map(&wd.tmA, dYp, H, P, 64, 64) || !make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
+    if (!make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
+    if (gather) {  // A = dY rows by token (its per-expert map copy is unused)
+      set_gather(wd, dY, T, k, H);
+      wd.tmA = wd.tmB;
+    } else if (!make_map(&wd.tmA, dYp, H, P, 64, 64)) {
+      return MOE_ERR_CUDA;
+    }
     if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, wd.tmA, wd.tmB, offsets, E,
                    maps + 2 * E) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -682,7 +761,10 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
     wd.out_ld = I;
     wd.out_expert_stride = static_cast<int64_t>(H) * I;
     const int64_t tiles = static_cast<int64_t>(E) * wd.m_tiles * wd.n_tiles;
-    if (int st = launch_gemm<kBwdWgrad>(wd, pair_grid(tiles, dev->num_sms), stream, kProfWgradDown)) return st;
+    const int grid = pair_grid(tiles, dev->num_sms);
+    if (int st = gather ? launch_gemm<kBwdWgrad, kGatherA>(wd, grid, stream, kProfWgradDown)
+                        : launch_gemm<kBwdWgrad>(wd, grid, stream, kProfWgradDown))
+      return st;
   }
   // 7. router logits gradient
   {
@@ -695,6 +777,28 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
       return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                  const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                  const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                  const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                  float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
+                        H, I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
+                    const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                    const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                    const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
+                    float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_bwd_impl(dY, X, true, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k, H,
+                        I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
 }
 
 size_t moe_router_workspace_bytes(int T, int H, int E) {

@@ -1,7 +1,9 @@
 """The whole expert layer as a sequence of the C-ABI calls.
 
 ``forward`` runs moe_route -> moe_permute -> moe_experts_fwd -> moe_combine
-and returns Y plus the saved state; ``backward`` runs moe_layer_bwd.
+and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. With
+gather=True (the default) the permute makes no Xp copy and the GEMMs read X
+and dY rows by token index (moe_experts_fwd_x / moe_layer_bwd_x).
 ``forward_from_x`` / ``backward_to_x`` also run the router Linear
 (moe_router_fwd in place of moe_route; moe_router_bwd after moe_layer_bwd,
 adding the router's share to dX and giving dW_r). All buffers are torch CUDA
@@ -30,38 +32,40 @@ class LayerState:
     O: torch.Tensor
     Y: torch.Tensor
     logits: torch.Tensor | None = None
+    X: torch.Tensor | None = None  # token-order input, kept for the gather-fused backward
 
 
 def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
-            save_gu: bool = True, bufs: dict | None = None, stream=None) -> LayerState:
+            save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = True) -> LayerState:
     """Y = combine(experts(permute(X, route(logits)))). ``bufs`` may hold
     preallocated outputs/workspaces (keys as in the returned state)."""
     b = bufs or {}
     T, E = logits.shape
     idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
-    return _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream)
+    return _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather)
 
 
 def forward_from_x(X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
-                   save_gu: bool = True, bufs: dict | None = None, stream=None) -> LayerState:
+                   save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = True) -> LayerState:
     """As ``forward``, with the logits computed on the GPU from the fp32
     router weight W_r [E, H] (moe_router_fwd)."""
     b = bufs or {}
     T, E = X.shape[0], W_r.shape[0]
     out = {n: b[n] for n in ("logits", "topk_idx", "topk_w", "probs") if b.get(n) is not None}
     r = B.moe_router_fwd(X, W_r, k, out=out, ws=b.get("router_ws"), stream=stream)
-    st = _experts_forward(T, E, k, r["topk_idx"], r["topk_w"], r["probs"], X, W_gu, W_d, save_gu, b, stream)
+    st = _experts_forward(T, E, k, r["topk_idx"], r["topk_w"], r["probs"], X, W_gu, W_d, save_gu, b, stream,
+                          gather)
     st.logits = r["logits"]
     return st
 
 
-def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream) -> LayerState:
-    perm = B.moe_permute(idx, E, X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
-    h, gu, O = B.moe_experts_fwd(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k, W_gu, W_d,
-                                 h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"), save_gu=save_gu,
-                                 stream=stream)
+def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather) -> LayerState:
+    perm = B.moe_permute(idx, E, None if gather else X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
+    h, gu, O = B.moe_experts_fwd(X if gather else perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k,
+                                 W_gu, W_d, h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"), save_gu=save_gu,
+                                 stream=stream, gather=gather)
     Y = B.moe_combine(O, perm["pair_pos"], T, k, Y=b.get("Y"), stream=stream)
-    return LayerState(T, E, k, idx, w, probs, perm, h, gu, O, Y)
+    return LayerState(T, E, k, idx, w, probs, perm, h, gu, O, Y, X=X if gather else None)
 
 
 def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, bufs: dict | None = None,
@@ -69,9 +73,10 @@ def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Te
     """dX, dW_gu, dW_d, dlogits for upstream gradient dY."""
     b = bufs or {}
     p = st.perm
-    return B.moe_layer_bwd(dY, p["Xp"], st.gu, st.h, st.probs, st.topk_idx, st.topk_w, p["offsets"],
-                           p["sorted_pair"], p["pair_pos"], st.T, st.E, st.k, W_gu, W_d,
-                           out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream)
+    gather = st.X is not None
+    return B.moe_layer_bwd(dY, st.X if gather else p["Xp"], st.gu, st.h, st.probs, st.topk_idx, st.topk_w,
+                           p["offsets"], p["sorted_pair"], p["pair_pos"], st.T, st.E, st.k, W_gu, W_d,
+                           out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream, gather=gather)
 
 
 def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor,
@@ -86,7 +91,8 @@ def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.
     return g
 
 
-def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False) -> dict:
+def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False,
+             gather: bool = True) -> dict:
     """Every output and workspace of one forward+backward, allocated once."""
     P = T * k
     bf = torch.bfloat16
@@ -98,8 +104,7 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
         perm=dict(counts=torch.empty(E, dtype=torch.int32, device=device),
                   offsets=torch.empty(E + 1, dtype=torch.int32, device=device),
                   sorted_pair=torch.empty(P, dtype=torch.int32, device=device),
-                  pair_pos=torch.empty(P, dtype=torch.int32, device=device),
-                  Xp=torch.empty(P, H, dtype=bf, device=device)),
+                  pair_pos=torch.empty(P, dtype=torch.int32, device=device)),
         perm_ws=torch.empty(max(lib.moe_permute_workspace_bytes(T, E, k), 1), dtype=torch.uint8, device=device),
         h=torch.empty(P, I, dtype=bf, device=device),
         gu=torch.empty(P, 2 * I, dtype=bf, device=device) if save_gu else None,
@@ -109,9 +114,11 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
                    dW_gu=torch.empty(E, 2 * I, H, dtype=bf, device=device),
                    dW_d=torch.empty(E, H, I, dtype=bf, device=device),
                    dlogits=torch.empty(T, E, dtype=torch.float32, device=device)),
-        bwd_ws=torch.empty(max(lib.moe_layer_bwd_workspace_bytes(T, E, k, H, I, 0 if save_gu else 1), 1),
-                           dtype=torch.uint8, device=device),
+        bwd_ws=torch.empty(max((lib.moe_layer_bwd_x_workspace_bytes if gather else lib.moe_layer_bwd_workspace_bytes)(
+            T, E, k, H, I, 0 if save_gu else 1), 1), dtype=torch.uint8, device=device),
     )
+    if not gather:
+        d["perm"]["Xp"] = torch.empty(P, H, dtype=bf, device=device)
     if router:
         d["logits"] = torch.empty(T, E, dtype=torch.float32, device=device)
         d["dW_r"] = torch.empty(E, H, dtype=torch.float32, device=device)

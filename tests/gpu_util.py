@@ -39,9 +39,9 @@ def to_dev(inp, dev="cuda"):
                 dY=None if inp.dY is None else inp.dY.to(dev))
 
 
-def run_layer(inp, k, backward=True, save_gu=True, stream=None):
+def run_layer(inp, k, backward=True, save_gu=True, stream=None, gather=True):
     d = to_dev(inp)
-    st = layer.forward(d["logits"], d["X"], d["W_gu"], d["W_d"], k, save_gu=save_gu, stream=stream)
+    st = layer.forward(d["logits"], d["X"], d["W_gu"], d["W_d"], k, save_gu=save_gu, stream=stream, gather=gather)
     grads = layer.backward(st, d["dY"], d["W_gu"], d["W_d"], stream=stream) if backward else None
     status = B.last_device_status(stream)
     assert status == 0, f"device status {B.status_str(status)}"
@@ -62,3 +62,15 @@ def oracle_full(inp, k):
     fwd = orc.layer_forward(inp.logits, inp.X, inp.W_gu, inp.W_d, k)
     bwd = orc.layer_backward(fwd, inp.dY, inp.X, inp.W_gu, inp.W_d, k) if inp.dY is not None else None
     return fwd, bwd
+
+
+def assert_same_results(a, ga, b, gb):
+    """Two runs of the layer (gathered and permuted operand loads) agree bit
+    for bit: the GEMMs see the same operand tiles in the same order."""
+    for name in ("Y", "h", "O"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    if a.gu is not None:
+        assert torch.equal(a.gu, b.gu), "gu"
+    if ga is not None:
+        for name in ("dX", "dW_gu", "dW_d", "dlogits"):
+            assert torch.equal(ga[name], gb[name]), name

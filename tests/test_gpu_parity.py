@@ -29,9 +29,13 @@ SHAPES = [
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "T%d_H%d_E%d_k%d_I%d" % s)
 def test_layer_matches_oracle(shape):
+    """Gathered operand loads (the default path) against the oracle, and bit
+    for bit against the path through the permuted copies Xp / dYp."""
     T, H, E, k, I = shape
     inp = small_inputs(T, H, E, k, I, seed=sum(shape))
     st, grads = U.run_layer(inp, k)
+    st_p, grads_p = U.run_layer(inp, k, gather=False)
+    U.assert_same_results(st, grads, st_p, grads_p)
     fwd, bwd = U.oracle_full(inp, k)
     U.check_routing_exact(st, fwd)
     U.assert_rel(U.to_np(st.h), fwd["h"], "h")
@@ -100,10 +104,11 @@ def test_route_permute_wide_and_narrow_E(E):
     assert (perm["counts"].cpu().numpy() == c).all()
 
 
-def test_recompute_gate_up_when_not_saved():
+@pytest.mark.parametrize("gather", [True, False])
+def test_recompute_gate_up_when_not_saved(gather):
     T, H, E, k, I = 500, 256, 8, 2, 192
     inp = small_inputs(T, H, E, k, I, seed=21)
-    st, grads = U.run_layer(inp, k, save_gu=False)
+    st, grads = U.run_layer(inp, k, save_gu=False, gather=gather)
     fwd, bwd = U.oracle_full(inp, k)
     assert st.gu is None
     for name in ("dX", "dW_gu", "dW_d", "dlogits"):
@@ -122,7 +127,8 @@ def test_non_default_stream():
     U.assert_rel(U.to_np(grads["dX"]), bwd["dX"], "dX")
 
 
-def test_empty_batch():
+@pytest.mark.parametrize("gather", [True, False])
+def test_empty_batch(gather):
     from routed_grouped_gemm_router_b200 import binding as B
     from routed_grouped_gemm_router_b200 import layer
     E, k, H, I = 8, 2, 64, 64
@@ -130,7 +136,7 @@ def test_empty_batch():
     X = torch.empty(0, H, dtype=torch.bfloat16, device="cuda")
     W_gu = torch.randn(E, 2 * I, H, device="cuda").bfloat16()
     W_d = torch.randn(E, H, I, device="cuda").bfloat16()
-    st = layer.forward(logits, X, W_gu, W_d, k)
+    st = layer.forward(logits, X, W_gu, W_d, k, gather=gather)
     assert st.Y.shape == (0, H) and (st.perm["counts"] == 0).all() and (st.perm["offsets"] == 0).all()
     grads = layer.backward(st, torch.empty(0, H, dtype=torch.bfloat16, device="cuda"), W_gu, W_d)
     assert (grads["dW_gu"] == 0).all() and (grads["dW_d"] == 0).all()
@@ -154,7 +160,7 @@ def test_backward_without_h():
     st, grads = U.run_layer(inp, k)
     d = U.to_dev(inp)
     p = st.perm
-    g2 = B.moe_layer_bwd(d["dY"], p["Xp"], st.gu, None, st.probs, st.topk_idx, st.topk_w, p["offsets"],
-                         p["sorted_pair"], p["pair_pos"], T, E, k, d["W_gu"], d["W_d"])
+    g2 = B.moe_layer_bwd(d["dY"], d["X"], st.gu, None, st.probs, st.topk_idx, st.topk_w, p["offsets"],
+                         p["sorted_pair"], p["pair_pos"], T, E, k, d["W_gu"], d["W_d"], gather=True)
     for name in ("dX", "dW_gu", "dW_d", "dlogits"):
         assert torch.equal(g2[name], grads[name]), name

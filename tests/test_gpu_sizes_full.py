@@ -50,3 +50,15 @@ def test_full_size_layer(name):
         else:
             U.assert_rel(U.to_np(grads["dW_gu"][e]), dgu, f"{name} dW_gu[{e}]")
             U.assert_rel(U.to_np(grads["dW_d"][e]), dd, f"{name} dW_d[{e}]")
+
+
+@pytest.mark.parametrize("name", ["qwen3-30b-a3b", "zipf-t32768", "zipf-t64"])
+def test_full_size_gathered_equals_permuted(name):
+    """At full size (long weight-gradient K for the hot experts, 20 empty
+    experts), the gathered operand loads give bit-identical results to the
+    loads from the permuted copies."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, seed=0, with_dy=True)
+    a, ga = U.run_layer(inp, wl.k)
+    b, gb = U.run_layer(inp, wl.k, gather=False)
+    U.assert_same_results(a, ga, b, gb)

@@ -490,6 +490,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // barrier of the stage (the third arrival it expects besides lane 0's
       // expect_tx and the other CTA's).
       constexpr bool kMN = kWgrad;
+      if (p.sorted_pair == nullptr || p.gsrc == nullptr || p.gather_rows < 1) {  // no row map: nothing to gather
+        if (lane == 0) report(MOE_ERR_DEVICE_CHECK);
+        *s_abort = 1;
+      }
       const int gk = p.gather_k > 0 ? p.gather_k : 1;
       const int gcols = p.gather_cols;
       const uint32_t leader_full0 = mapa_shared(smem_u32(&full_bar[0]), 0);

@@ -43,13 +43,9 @@
 namespace moe {
 
 enum GemmKind : int { kFwdGateUp = 0, kFwdDown = 1, kBwdDgradDown = 2, kBwdDgradGateUp = 3, kBwdWgrad = 4 };
-// Which operand, if any, the producer warp gathers itself with 16-byte
-// cp.async copies from a token-order tensor (row = sorted_pair[r] /
-// gather_k) instead of loading a permuted copy with TMA.
+// Which operand, if any, is read with row-gather TMA from a token-order
+// tensor (tmG; row = sorted_pair[r] / gather_k) instead of a permuted copy.
 enum GatherMode : int { kNoGather = 0, kGatherA = 1, kGatherB = 2 };
-// Gathered stages are signalled this many stages after they are issued (the
-// copies of the older stage have landed by then).
-constexpr int kGatherLag = 2;
 
 constexpr int kBM = 256;        // rows of a pair tile
 constexpr int kBMc = 128;       // rows per CTA
@@ -102,6 +98,7 @@ constexpr int kStageWarpBytes = 32 * kStageStrideBytes;
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmG;                 // gathered operand: token-order [gather_rows, gather_cols], box 64 x 1
   const CUtensorMap* expert_maps;  // wgrad: [2][E] maps (A then B) clipped at each segment end
   const int32_t* offsets;      // [E+1] expert segment bounds in the permuted rows
   const int32_t* sorted_pair;  // [P]
@@ -121,7 +118,6 @@ struct GemmParams {
   uint16_t* gu;               // FwdGateUp: optional g|u save; BwdDgradDown: g|u input
   uint16_t* hw_out;           // BwdDgradDown: w_q * h
   float* dw_part;             // BwdDgradDown: [P, kDwSlotsPerNTile * n_tiles] partial routing-weight grads
-  const uint16_t* gsrc;       // gathered operand: token-order [gather_rows, gather_cols] bf16
   int gather_k;               // pair id -> token: q / gather_k
   int gather_rows;
   int gather_cols;
@@ -129,8 +125,7 @@ struct GemmParams {
 
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
   return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes + kNumBarriers * 8 + 16 +
-         2 * static_cast<size_t>(E + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * kStageWarpBytes +
-         2 * 128 * 4 /* gathered rows' token ids */;
+         2 * static_cast<size_t>(E + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * kStageWarpBytes;
 }
 
 struct TileInfo {
@@ -299,7 +294,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
   int* s_tstart = s_off + (p.E + 1);
   uint8_t* s_stage = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 15) & ~uintptr_t(15));
-  int* s_gtok = reinterpret_cast<int*>(s_stage + kEpiWarps * kStageWarpBytes);  // [2][128] token ids
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -310,8 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // ------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      // gathered stages: also one arrival per CTA once its copies have landed
-      mbar_init(&full_bar[s], GATHER != kNoGather ? 3 : 1);
+      mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -325,6 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
+    if constexpr (GATHER != kNoGather) tma_prefetch_desc(&p.tmG);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, kTmemCols);
@@ -474,58 +468,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     if constexpr (GATHER != kNoGather) {
       // ------------------------------------- producer with a gathered operand
-      // Lane 0 loads the other operand with TMA exactly as above (both CTAs'
-      // bytes on the even CTA's full barrier). All 32 lanes copy the gathered
-      // operand's tile with 16-byte cp.async straight into its 128-byte
-      // swizzled layout. K-major A (row-grouped kinds): instruction j covers
-      // rows 4j..4j+3 of the CTA's 128 tile rows, lane l the 16-byte chunk
-      // l%8 of row 4j+l/8. MN-major operand (weight gradients): instruction j
-      // covers K rows 2j and 2j+1, lane l the 16-byte piece l%16 of the CTA's
-      // 128 MN columns. Each instruction therefore reads four whole 128-byte
-      // lines. Rows past the segment end read token 0 (their outputs are
-      // masked, or the other operand is zero there); columns past the tensor
-      // are zero-filled. A stage's copies form one commit group; kGatherLag
-      // stages later the warp waits for that group, fences the generic proxy
-      // against the async proxy, and lane 0 arrives on the even CTA's full
-      // barrier of the stage (the third arrival it expects besides lane 0's
-      // expect_tx and the other CTA's).
+      // Lane 0 loads the other operand with TMA exactly as above. The
+      // gathered operand's tile is loaded by all 32 lanes with row-gather
+      // TMA (four 128-byte rows per load, 512 bytes apart in the 128-byte
+      // swizzled tile), completing on the even CTA's full barrier like every
+      // other load of the pair. K-major A (row-grouped kinds): lane l loads
+      // rows 4l..4l+3 of the CTA's 128 tile rows at K block kb. MN-major
+      // operand (weight gradients): lane l loads K rows 4(l%16)..+3 of the
+      // block into MN chunk l/16 of the CTA's 128 MN columns; a chunk wholly
+      // past the tensor's columns (it only feeds masked outputs) reads chunk
+      // 0 instead. Rows past the segment end read token 0: their outputs are
+      // masked, or the other operand is zero there.
       constexpr bool kMN = kWgrad;
-      if (p.sorted_pair == nullptr || p.gsrc == nullptr || p.gather_rows < 1) {  // no row map: nothing to gather
+      if (p.sorted_pair == nullptr || p.gather_rows < 1) {  // no row map: nothing to gather
         if (lane == 0) report(MOE_ERR_DEVICE_CHECK);
         *s_abort = 1;
       }
       const int gk = p.gather_k > 0 ? p.gather_k : 1;
       const int gcols = p.gather_cols;
-      const uint32_t leader_full0 = mapa_shared(smem_u32(&full_bar[0]), 0);
       auto tok_of = [&](int32_t q) {
         const int t = q / gk;
         return t < 0 ? 0 : (t >= p.gather_rows ? p.gather_rows - 1 : t);
       };
-      int stage = 0, sig_stage = 0, pending = 0, issued = 0;
-      uint32_t phase = 0;
-      auto signal_oldest = [&]() {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_full0 + sig_stage * 8);
-        if (++sig_stage == kStages) sig_stage = 0;
-        --pending;
-      };
-      // row-grouped: pair ids of this CTA's 4 rows per lane (rows lane + 32m),
-      // requested one tile ahead
-      int32_t q_nxt[4] = {0, 0, 0, 0};
-      auto load_tile_pairs = [&](int t, int32_t (&q)[4]) {
+      auto tile_pairs = [&](int t, int32_t (&q)[4]) {
         const TileInfo tn = decode_tile<KIND>(t, p, s_off, s_tstart);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const int r = static_cast<int>(rank) * kBMc + lane + 32 * m;
+          const int r = static_cast<int>(rank) * kBMc + 4 * lane + m;
           q[m] = r < tn.rows ? __ldg(p.sorted_pair + tn.row0 + r) : 0;
         }
       };
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      int32_t q_nxt[4] = {0, 0, 0, 0};
       if constexpr (!kMN) {
-        if (pair < total_tiles) load_tile_pairs(pair, q_nxt);
+        if (pair < total_tiles && !*s_abort) tile_pairs(pair, q_nxt);
       }
-      int tile_iter = 0;
-      for (int t = pair; t < total_tiles && !__any_sync(0xffffffffu, *s_abort != 0); t += num_pairs, ++tile_iter) {
+      for (int t = pair; t < total_tiles && !__any_sync(0xffffffffu, *s_abort != 0); t += num_pairs) {
         const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
         if constexpr (kWgrad) {
           if (ti.num_kb == 0) continue;
@@ -534,39 +513,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tensormap_acquire(p.expert_maps + p.E + ti.e);
           }
         }
-        int* tokbuf = s_gtok + (tile_iter & 1) * 128;
-        int32_t qm0a = 0, qm0b = 0, qm1a = 0, qm1b = 0;  // MN: pair ids of K blocks kb, kb+1
-        auto load_block_pairs = [&](int kb, int32_t& qa, int32_t& qb) {
-          const int r = kb * kBK + lane;
-          qa = (kb < ti.num_kb && r < ti.rows) ? __ldg(p.sorted_pair + ti.row0 + r) : 0;
-          qb = (kb < ti.num_kb && r + 32 < ti.rows) ? __ldg(p.sorted_pair + ti.row0 + r + 32) : 0;
+        // gathered pair ids: the tile's (row-grouped; requested one tile
+        // ahead) or those of K blocks kb and kb+1 (wgrad; two blocks ahead)
+        int32_t q_cur[4] = {0, 0, 0, 0}, q_k1[4] = {0, 0, 0, 0}, q_k2[4] = {0, 0, 0, 0};
+        auto block_pairs = [&](int kb, int32_t (&q)[4]) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int r = kb * kBK + 4 * (lane & 15) + m;
+            q[m] = (kb < ti.num_kb && r < ti.rows) ? __ldg(p.sorted_pair + ti.row0 + r) : 0;
+          }
         };
         if constexpr (!kMN) {
-          int32_t q_cur[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) q_cur[m] = q_nxt[m];
-          if (t + num_pairs < total_tiles) load_tile_pairs(t + num_pairs, q_nxt);
-          __syncwarp();
-#pragma unroll
-          for (int m = 0; m < 4; ++m) tokbuf[lane + 32 * m] = tok_of(q_cur[m]);
-          __syncwarp();
+          if (t + num_pairs < total_tiles) tile_pairs(t + num_pairs, q_nxt);
         } else {
-          load_block_pairs(0, qm0a, qm0b);
-          load_block_pairs(1, qm1a, qm1b);
+          block_pairs(0, q_k1);
+          block_pairs(1, q_k2);
         }
         bool ok = true;
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           if constexpr (kMN) {
-            // token ids of this block's 64 K rows (buffer kb & 1; its readers
-            // from block kb-2 are past the __syncwarp below)
-            int* tb = s_gtok + (kb & 1) * 128;
-            __syncwarp();
-            tb[lane] = tok_of(qm0a);
-            tb[lane + 32] = tok_of(qm0b);
-            qm0a = qm1a;
-            qm0b = qm1b;
-            load_block_pairs(kb + 2, qm1a, qm1b);
-            __syncwarp();
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              q_cur[m] = q_k1[m];
+              q_k1[m] = q_k2[m];
+            }
+            block_pairs(kb + 2, q_k2);
           }
           if (!warp_wait(&empty_bar[stage], phase ^ 1u)) {
             if (lane == 0) report(MOE_ERR_TIMEOUT);
@@ -574,46 +547,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (lane == 0) {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (kStageBytes - kATileBytes));
-            issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes,
-                  mapa_shared(smem_u32(&full_bar[stage]), 0));
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
+            issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes, fb);
           }
-          const int kx = kb * kBK;
-          if constexpr (!kMN) {
-            const int c = lane & 7;
-            const uint32_t nbytes = (kx + 8 * c < gcols) ? 16u : 0u;
-            const int col = nbytes ? kx + 8 * c : 0;
-            const uint32_t dst0 = smem_u32(sA + stage * kATileBytes);
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-              const int i = 4 * j + (lane >> 3);
-              const uint16_t* src = p.gsrc + static_cast<int64_t>(tokbuf[i]) * gcols + col;
-              cp_async_16(dst0 + i * 128 + ((c ^ (i & 7)) << 4), src, nbytes);
-            }
-          } else {
-            const int* tb = s_gtok + (kb & 1) * 128;
-            const int pp = lane & 15;
-            const int mn0 = (GATHER == kGatherA ? ti.m_blk * kBM : ti.n_blk * kBN) + static_cast<int>(rank) * 128;
-            const int colp = mn0 + 8 * pp;
-            const uint32_t nbytes = colp < gcols ? 16u : 0u;
-            const int col = nbytes ? colp : 0;
-            uint8_t* g_tile = GATHER == kGatherA ? sA + stage * kATileBytes : sB + stage * kBTileBytes;
-            const uint32_t dst0 = smem_u32(g_tile) + 8192 * (pp >> 3);
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-              const int k = 2 * j + (lane >> 4);
-              const uint16_t* src = p.gsrc + static_cast<int64_t>(tb[k]) * gcols + col;
-              cp_async_16(dst0 + k * 128 + (((pp & 7) ^ (k & 7)) << 4), src, nbytes);
-            }
+          uint8_t* g_tile = (GATHER == kGatherA) ? sA + stage * kATileBytes : sB + stage * kBTileBytes;
+          int gx = kb * kBK, goff = 512 * lane;
+          if constexpr (kMN) {
+            const int chunk = lane >> 4;
+            gx = (GATHER == kGatherA ? ti.m_blk * kBM : ti.n_blk * kBN) + static_cast<int>(rank) * kBMc + 64 * chunk;
+            if (gx >= gcols) gx = 0;
+            goff = 8192 * chunk + 512 * (lane & 15);
           }
-          cp_async_commit();
-          ++pending;
+          tma_gather4_pair(g_tile + goff, &p.tmG, fb, gx, tok_of(q_cur[0]), tok_of(q_cur[1]), tok_of(q_cur[2]),
+                           tok_of(q_cur[3]));
           ++issued;
-          if (pending > kGatherLag) {
-            cp_async_wait<kGatherLag>();
-            signal_oldest();
-          }
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -621,10 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
       }
-      // every copy has landed and every issued stage is signalled before the
-      // CTA leaves
-      cp_async_wait<0>();
-      while (pending > 0) signal_oldest();
+      // no load of the pair may still be in flight when it leaves
       if (lane == 0 && rank == 0) {
         const int inflight = issued < kStages ? issued : kStages;
         for (int i = 0; i < inflight; ++i) {

@@ -223,14 +223,16 @@ inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
 }
 
 // The gathered operand of a GEMM: token-order rows [T, H] picked by
-// sorted_pair[r] / k. Its tensor map is not loaded from; a valid map is kept
-// in its place for the kernel's descriptor prefetch.
-void set_gather(GemmParams& g, const moe_bf16* src, const int32_t* sorted_pair, int T, int k, int H) {
-  g.gsrc = src;
+// sorted_pair[r] / k, read through a row-gather map (64-column boxes one row
+// high). The operand's own tensor map is not loaded from; the caller keeps a
+// valid map in its place for the kernel's descriptor prefetch.
+bool set_gather(GemmParams& g, const moe_bf16* src, const int32_t* sorted_pair, int T, int k, int H) {
+  if (!make_map(&g.tmG, src, H, T, 64, 1)) return false;
   g.sorted_pair = sorted_pair;  // the gathering producer maps rows to tokens through it
   g.gather_k = k;
   g.gather_rows = T;
   g.gather_cols = H;
+  return true;
 }
 
 GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
@@ -513,7 +515,7 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   GemmParams gu = base_params(E, P, offsets);
   if (!make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
   if (gather) {
-    set_gather(gu, src, sorted_pair, T, k, H);
+    if (!set_gather(gu, src, sorted_pair, T, k, H)) return MOE_ERR_CUDA;
     gu.tmA = gu.tmB;
   } else if (!make_map(&gu.tmA, Xp, H, P, 64, 128)) {
     return MOE_ERR_CUDA;
@@ -642,7 +644,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     GemmParams rc = base_params(E, P, offsets);
     if (!make_map(&rc.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
     if (gather) {
-      set_gather(rc, src, sorted_pair, T, k, H);
+      if (!set_gather(rc, src, sorted_pair, T, k, H)) return MOE_ERR_CUDA;
       rc.tmA = rc.tmB;
     } else if (!make_map(&rc.tmA, Xp, H, P, 64, 128)) {
       return MOE_ERR_CUDA;
@@ -666,7 +668,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     GemmParams bd = base_params(E, P, offsets);
     if (!make_map(&bd.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 64)) return MOE_ERR_CUDA;
     if (gather) {
-      set_gather(bd, dY, sorted_pair, T, k, H);
+      if (!set_gather(bd, dY, sorted_pair, T, k, H)) return MOE_ERR_CUDA;
       bd.tmA = bd.tmB;
     } else if (!make_map(&bd.tmA, dYp, H, P, 64, 128)) {
       return MOE_ERR_CUDA;
@@ -717,7 +719,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     GemmParams wg = base_params(E, P, offsets);
     if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64)) return MOE_ERR_CUDA;
     if (gather) {  // B = X rows by token (its per-expert map copy is unused)
-      set_gather(wg, src, sorted_pair, T, k, H);
+      if (!set_gather(wg, src, sorted_pair, T, k, H)) return MOE_ERR_CUDA;
       wg.tmB = wg.tmA;
     } else if (!make_map(&wg.tmB, Xp, H, P, 64, 64)) {
       return MOE_ERR_CUDA;
@@ -744,7 +746,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     GemmParams wd = base_params(E, P, offsets);
     if (!make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
     if (gather) {  // A = dY rows by token (its per-expert map copy is unused)
-      set_gather(wd, dY, sorted_pair, T, k, H);
+      if (!set_gather(wd, dY, sorted_pair, T, k, H)) return MOE_ERR_CUDA;
       wd.tmA = wd.tmB;
     } else if (!make_map(&wd.tmA, dYp, H, P, 64, 64)) {
       return MOE_ERR_CUDA;

@@ -281,6 +281,7 @@ def workload_config(wl, args):
                         f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else "")
                         + (" + router Linear (fp32, on the GPU)" if getattr(args, "router_linear", False) else ""),
             "router_linear": bool(getattr(args, "router_linear", False)),
+            "gather_fused": bool(getattr(args, "gather_fused", False)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -293,6 +294,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qwen3-30b-a3b", choices=sorted(WORKLOADS))
     ap.add_argument("--forward-only", action="store_true")
+    ap.add_argument("--gather-fused", action="store_true",
+                    help="GEMMs read X / dY rows by token (no Xp / dYp copies) instead of the permuted copies")
     ap.add_argument("--router-linear", action="store_true",
                     help="include the router Linear (logits = X W_r^T and its backward) in the step")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -335,17 +338,18 @@ def main():
     rl = args.router_linear
     if rl and wl.zipf_s:
         ap.error("--router-linear: the stress workloads' logit bias has no router-weight form")
-    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl)
+    gf = args.gather_fused
+    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl, gather=gf)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
         if rl:
-            st = layer.forward_from_x(X, W_r, W_gu, W_d, wl.k, bufs=bufs)
+            st = layer.forward_from_x(X, W_r, W_gu, W_d, wl.k, bufs=bufs, gather=gf)
             if wl.backward:
                 layer.backward_to_x(st, dY, X, W_r, W_gu, W_d, bufs=bufs)
             return
-        st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs)
+        st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs, gather=gf)
         if wl.backward:
             layer.backward(st, dY, W_gu, W_d, bufs=bufs)
 
@@ -462,11 +466,11 @@ def main():
                 stream.wait_event(ev_in[b])
                 stream.wait_event(ev_copied[b])
                 if rl:
-                    st = layer.forward_from_x(din[b]["X"], W_r, W_gu, W_d, wl.k, bufs=obufs[b])
+                    st = layer.forward_from_x(din[b]["X"], W_r, W_gu, W_d, wl.k, bufs=obufs[b], gather=gf)
                     if wl.backward:
                         g = layer.backward_to_x(st, din[b]["dY"], din[b]["X"], W_r, W_gu, W_d, bufs=obufs[b])
                 else:
-                    st = layer.forward(din[b]["logits"], din[b]["X"], W_gu, W_d, wl.k, bufs=obufs[b])
+                    st = layer.forward(din[b]["logits"], din[b]["X"], W_gu, W_d, wl.k, bufs=obufs[b], gather=gf)
                     if wl.backward:
                         g = layer.backward(st, din[b]["dY"], W_gu, W_d, bufs=obufs[b])
                 ev_used[b].record(stream)

@@ -2,8 +2,10 @@
 
 ``forward`` runs moe_route -> moe_permute -> moe_experts_fwd -> moe_combine
 and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. With
-gather=True (the default) the permute makes no Xp copy and the GEMMs read X
-and dY rows by token index (moe_experts_fwd_x / moe_layer_bwd_x).
+gather=True the permute makes no Xp copy and the GEMMs read X and dY rows by
+token index (moe_experts_fwd_x / moe_layer_bwd_x): no Xp / dYp buffers
+(2 x T*k*H bf16 less memory), but the row-gather loads make those GEMMs
+slower, so the default keeps the permuted copies.
 ``forward_from_x`` / ``backward_to_x`` also run the router Linear
 (moe_router_fwd in place of moe_route; moe_router_bwd after moe_layer_bwd,
 adding the router's share to dX and giving dW_r). All buffers are torch CUDA
@@ -36,7 +38,7 @@ class LayerState:
 
 
 def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
-            save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = True) -> LayerState:
+            save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = False) -> LayerState:
     """Y = combine(experts(permute(X, route(logits)))). ``bufs`` may hold
     preallocated outputs/workspaces (keys as in the returned state)."""
     b = bufs or {}
@@ -46,7 +48,7 @@ def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torc
 
 
 def forward_from_x(X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
-                   save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = True) -> LayerState:
+                   save_gu: bool = True, bufs: dict | None = None, stream=None, gather: bool = False) -> LayerState:
     """As ``forward``, with the logits computed on the GPU from the fp32
     router weight W_r [E, H] (moe_router_fwd)."""
     b = bufs or {}
@@ -92,7 +94,7 @@ def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.
 
 
 def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False,
-             gather: bool = True) -> dict:
+             gather: bool = False) -> dict:
     """Every output and workspace of one forward+backward, allocated once."""
     P = T * k
     bf = torch.bfloat16

@@ -39,7 +39,7 @@ def to_dev(inp, dev="cuda"):
                 dY=None if inp.dY is None else inp.dY.to(dev))
 
 
-def run_layer(inp, k, backward=True, save_gu=True, stream=None, gather=True):
+def run_layer(inp, k, backward=True, save_gu=True, stream=None, gather=False):
     d = to_dev(inp)
     st = layer.forward(d["logits"], d["X"], d["W_gu"], d["W_d"], k, save_gu=save_gu, stream=stream, gather=gather)
     grads = layer.backward(st, d["dY"], d["W_gu"], d["W_d"], stream=stream) if backward else None

@@ -29,13 +29,13 @@ SHAPES = [
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "T%d_H%d_E%d_k%d_I%d" % s)
 def test_layer_matches_oracle(shape):
-    """Gathered operand loads (the default path) against the oracle, and bit
-    for bit against the path through the permuted copies Xp / dYp."""
+    """The default path (permuted copies Xp / dYp) against the oracle, and the
+    gather-fused path bit for bit against it."""
     T, H, E, k, I = shape
     inp = small_inputs(T, H, E, k, I, seed=sum(shape))
     st, grads = U.run_layer(inp, k)
-    st_p, grads_p = U.run_layer(inp, k, gather=False)
-    U.assert_same_results(st, grads, st_p, grads_p)
+    st_g, grads_g = U.run_layer(inp, k, gather=True)
+    U.assert_same_results(st_g, grads_g, st, grads)
     fwd, bwd = U.oracle_full(inp, k)
     U.check_routing_exact(st, fwd)
     U.assert_rel(U.to_np(st.h), fwd["h"], "h")
@@ -160,7 +160,7 @@ def test_backward_without_h():
     st, grads = U.run_layer(inp, k)
     d = U.to_dev(inp)
     p = st.perm
-    g2 = B.moe_layer_bwd(d["dY"], d["X"], st.gu, None, st.probs, st.topk_idx, st.topk_w, p["offsets"],
-                         p["sorted_pair"], p["pair_pos"], T, E, k, d["W_gu"], d["W_d"], gather=True)
+    g2 = B.moe_layer_bwd(d["dY"], p["Xp"], st.gu, None, st.probs, st.topk_idx, st.topk_w, p["offsets"],
+                         p["sorted_pair"], p["pair_pos"], T, E, k, d["W_gu"], d["W_d"])
     for name in ("dX", "dW_gu", "dW_d", "dlogits"):
         assert torch.equal(g2[name], grads[name]), name

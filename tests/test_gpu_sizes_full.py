@@ -59,6 +59,6 @@ def test_full_size_gathered_equals_permuted(name):
     loads from the permuted copies."""
     wl = WORKLOADS[name]
     inp = make_inputs(wl, seed=0, with_dy=True)
-    a, ga = U.run_layer(inp, wl.k)
-    b, gb = U.run_layer(inp, wl.k, gather=False)
+    a, ga = U.run_layer(inp, wl.k, gather=True)
+    b, gb = U.run_layer(inp, wl.k)
     U.assert_same_results(a, ga, b, gb)

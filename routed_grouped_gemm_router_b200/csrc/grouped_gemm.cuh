@@ -820,9 +820,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      // The warp's TMEM reads are complete (tcgen05.wait::ld); the arrival
+      // only hands the accumulator buffer back to the MMA issuer, so it does
+      // not wait for the tile's global stores to drain.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);
+#ifndef MOE_TEMPTY_RELAXED
+#define MOE_TEMPTY_RELAXED 1
+#endif
+      if (lane == 0) {
+        if (MOE_TEMPTY_RELAXED) mbar_arrive_cluster_relaxed(leader_tempty0 + acc * 8);
+        else mbar_arrive_cluster(leader_tempty0 + acc * 8);
+      }
       ++tcount;
     }
   }

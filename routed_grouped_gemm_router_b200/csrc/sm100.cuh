@@ -209,6 +209,13 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// The same arrival without release semantics: it does not wait for the
+// thread's earlier memory writes to become visible. For signals that order
+// only execution (an accumulator buffer whose tcgen05.ld reads have already
+// completed), not data.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 
 // 2-D tiled TMA load into this CTA's shared memory whose completion bytes are
 // counted on an mbarrier of either CTA of the pair (cluster address).

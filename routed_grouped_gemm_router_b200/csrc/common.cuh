@@ -56,23 +56,34 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
 // Launches `kernel` on stream `s` with programmatic stream serialisation, so
 // its set-up may overlap the tail of the previous kernel on the stream (the
 // kernel itself waits for that kernel's results, see griddep_wait).
+// cluster_x > 1 launches clusters of cluster_x CTAs along x.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args&&... args) {
+inline cudaError_t launch_pdl_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                        cudaStream_t s, unsigned cluster_x, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
 #ifndef MOE_PDL
 #define MOE_PDL 1
 #endif
   attr[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster_x > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  return launch_pdl_clustered(kernel, grid, block, smem, s, 1u, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

@@ -329,6 +329,24 @@ int launch_router_gemm(const RouterGemmParams& p, cudaStream_t s, int slot) {
   return launch_status();
 }
 
+// Logits + routing in one launch (clusters of two CTAs per 128-token tile).
+#ifndef MOE_ROUTER_FUSED_ROUTE
+#define MOE_ROUTER_FUSED_ROUTE 1
+#endif
+constexpr bool kRouterFusedRoute = MOE_ROUTER_FUSED_ROUTE != 0;
+template <int KMAX>
+int launch_router_route(const RouterGemmParams& p, cudaStream_t s) {
+  const size_t smem = rg_smem_bytes(p.bn, p.stages, p.N);
+  if (cudaFuncSetAttribute(router_gemm_kernel<kRgLogitsRoute, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ProfScope ps(kProfRouterLogits, s);
+  if (launch_pdl_clustered(router_gemm_kernel<kRgLogitsRoute, KMAX>, dim3(2 * p.m_tiles), dim3(kRgThreads), smem, s,
+                           2u, p) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_status();
+}
+
 int launch_split3(const float* src, int64_t rows, int cols, int src_ld, int dst_ld, int64_t term_rows,
                   uint16_t* dst, int num_sms, cudaStream_t s, int slot) {
   const int64_t n = rows * cols;
@@ -843,6 +861,20 @@ int moe_router_fwd(const moe_bf16* X, const float* W_r, int T, int H, int E, int
   p.out_split_stride = int64_t(T) * E8;
   if (!make_map(&p.tmA, X, H, T, 64, kRgBM) || !make_map(&p.tmB, w3, H, 3 * int64_t(E), 64, p.bn))
     return MOE_ERR_CUDA;
+  if (E <= kRgRouteMaxE && k <= 32 && kRouterFusedRoute) {
+    // one kernel: K split over the two CTAs of a cluster, routing in the epilogue
+    p.splits = 2;
+    p.n_tiles = 1;
+    p.stages = 4;
+    p.k = k;
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    p.probs = probs;
+    p.logits = logits;
+    if (k <= 8) return launch_router_route<8>(p, stream);
+    if (k <= 16) return launch_router_route<16>(p, stream);
+    return launch_router_route<32>(p, stream);
+  }
   if (int st = launch_router_gemm<kRgLogits>(p, stream, kProfRouterLogits)) return st;
   ProfScope ps(kProfRoute, stream);
   if (launch_route(nullptr, T, E, k, topk_idx, topk_w, probs, stream, part, p.splits, E8, int64_t(T) * E8, logits) !=

@@ -32,6 +32,10 @@ enum RouterGemmKind : int {
   kRgLogits = 0,  // out[split][t][e]   = sum_k X[t,k] W3[term*E + e, k]           (fp32 partials)
   kRgWgrad = 1,   // out[split][e][h]   = sum_t dl3[term*T + t, e] X[t, h]        (fp32 partials of dW_r)
   kRgDgrad = 2,   // dX[t][h] += sum_e dl3[a*T + t, e] W3[b*E + e, h], (a,b) pairs (bf16 in/out)
+  // logits as kRgLogits, K split over the two CTAs of a cluster; the odd CTA
+  // adds its partial into the even CTA's shared memory, which then routes
+  // (softmax, top-k, renormalisation) in the epilogue (E <= 128, k <= KMAX)
+  kRgLogitsRoute = 3,
 };
 
 constexpr int kRgBM = 128;
@@ -65,7 +69,19 @@ struct RouterGemmParams {
   int64_t out_split_stride;
   uint16_t* dx;      // bf16 in/out (dgrad)
   int dx_ld;
+  // kRgLogitsRoute outputs (logits and probs may be null)
+  int k;
+  int32_t* topk_idx;
+  float* topk_w;
+  float* probs;
+  float* logits;
 };
+
+// Fused routing: row stride (in floats) of the [E][128] logits buffer in
+// shared memory; 129 keeps both row-wise and column-wise accesses free of
+// bank conflicts.
+constexpr int kRgLgStride = 129;
+constexpr int kRgRouteMaxE = 128;
 
 __host__ __device__ inline int rg_b_tile_bytes(int bn) { return bn * kRgBK * 2; }
 __host__ __device__ inline int rg_tmem_cols(int bn) {
@@ -76,9 +92,9 @@ __host__ __device__ inline int rg_tmem_cols(int bn) {
 // The epilogue's staging blocks (4 warps x 4 KiB) reuse stage 0's A tile: a
 // CTA computes one tile, so every load and MMA is finished when its epilogue
 // starts.
-inline size_t rg_smem_bytes(int bn, int stages) {
+inline size_t rg_smem_bytes(int bn, int stages, int lg_rows = 0) {
   return 1024 /* alignment slack */ + static_cast<size_t>(stages) * (kRgATileBytes + rg_b_tile_bytes(bn)) +
-         256 /* barriers, TMEM slot, flags */;
+         256 /* barriers, TMEM slot, flags */ + static_cast<size_t>(lg_rows) * kRgLgStride * 4;
 }
 static_assert(4 * kRgStageWarpBytes <= kRgATileBytes, "epilogue staging must fit in one A tile");
 
@@ -106,8 +122,9 @@ __device__ __forceinline__ bool rg_warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int KIND>
+template <int KIND, int KMAX = 1>
 __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid_constant__ RouterGemmParams p) {
+  constexpr bool kRoute = (KIND == kRgLogitsRoute);
   constexpr bool kAMN = (KIND == kRgWgrad);  // A = X^T: M (hidden) contiguous
   constexpr bool kBMN = (KIND != kRgLogits); // B = dl3 (wgrad) or W3 (dgrad): N contiguous
   constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
@@ -130,16 +147,19 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
   uint64_t* drain_bar = bars + 2 * kRgMaxStages + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kRgMaxStages + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  float* s_lg = reinterpret_cast<float*>(s_tmem + 16);  // kRgLogitsRoute: logits [E][kRgLgStride]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t tmem_cols = static_cast<uint32_t>(rg_tmem_cols(bn));
 
-  // unit -> (M tile, N tile, K range); the splits of one output tile are adjacent
+  // unit -> (M tile, N tile, K range); the splits of one output tile are
+  // adjacent (for kRgLogitsRoute they are the two CTAs of a cluster)
   const int unit = blockIdx.x;
-  const int split = unit % p.splits;
-  const int n_blk = (unit / p.splits) % p.n_tiles;
-  const int m_blk = unit / (p.splits * p.n_tiles);
+  const uint32_t crank = kRoute ? cluster_ctarank() : 0u;
+  const int split = kRoute ? static_cast<int>(crank) : unit % p.splits;
+  const int n_blk = kRoute ? 0 : (unit / p.splits) % p.n_tiles;
+  const int m_blk = kRoute ? (unit >> 1) : unit / (p.splits * p.n_tiles);
   const int m0 = m_blk * kRgBM;
   const int n0 = n_blk * bn;
   const int64_t G = static_cast<int64_t>(p.n_terms) * p.nkb;
@@ -189,7 +209,7 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
         uint8_t* a_dst = sA + stage * kRgATileBytes;
         uint8_t* b_dst = sB + stage * b_bytes;
         mbar_arrive_expect_tx(fb, static_cast<uint32_t>(kRgATileBytes + b_bytes));
-        if constexpr (KIND == kRgLogits) {
+        if constexpr (KIND == kRgLogits || kRoute) {
           tma_load_2d(a_dst, &p.tmA, fb, kx, m0);
           tma_load_2d(b_dst, &p.tmB, fb, kx, term * p.term_rows_b + n0);
         } else if constexpr (KIND == kRgWgrad) {
@@ -292,7 +312,27 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
       *s_abort = 1;
     }
     tc_fence_after();
-    if (ok && !*s_abort && KIND == kRgDgrad) {
+    if (kRoute && ok && !*s_abort && crank == 1) {
+      // odd CTA of the cluster: its fp32 partial goes into the even CTA's
+      // logits buffer (element [e][row]; lanes write consecutive rows)
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
+      const uint32_t peer_lg = mapa_shared(smem_u32(s_lg), 0);
+      const int r = sub * 32 + lane;
+#pragma unroll 1
+      for (int ch = 0; ch < (bn + 31) / 32; ++ch) {
+        if (ch * 32 >= p.N) break;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + ch * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = ch * 32 + j;
+          if (e < p.N) st_shared_cluster_f32(peer_lg + static_cast<uint32_t>(e * kRgLgStride + r) * 4u, __uint_as_float(v[j]));
+        }
+      }
+    } else if (kRoute) {
+      // even CTA: routes after the cluster barrier below
+    } else if (ok && !*s_abort && KIND == kRgDgrad) {
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
       const int row0 = m0 + sub * 32;
 #pragma unroll
@@ -371,6 +411,107 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
       }
     }
     tc_fence_before();
+  }
+
+  if constexpr (kRoute) {
+    // ------------------------------------------ routing (even CTA of the pair)
+    __syncthreads();
+    __syncwarp();
+    cluster_sync_all();  // the odd CTA's partial has landed in s_lg
+    if (crank == 0 && warp >= 2 && !*s_abort) {
+      const int sub = warp & 3;
+      const int r = sub * 32 + lane;  // row of the tile owned by this thread
+      const int t = m0 + r;
+      const int E = p.N;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
+      tc_fence_after();
+      // logits = (even CTA's partial) + (odd CTA's partial), fp32
+#pragma unroll 1
+      for (int ch = 0; ch < (bn + 31) / 32; ++ch) {
+        if (ch * 32 >= E) break;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + ch * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = ch * 32 + j;
+          if (e < E) s_lg[e * kRgLgStride + r] = __uint_as_float(v[j]) + s_lg[e * kRgLgStride + r];
+        }
+      }
+      __syncwarp();
+      if (p.logits != nullptr) {  // the warp's 32 rows, coalesced
+        for (int i = 0; i < 32; ++i) {
+          const int row = sub * 32 + i;
+          if (m0 + row >= p.M) break;
+          for (int e = lane; e < E; e += 32)
+            p.logits[static_cast<int64_t>(m0 + row) * E + e] = s_lg[e * kRgLgStride + row];
+        }
+      }
+      // max and top-k (logit descending, lower expert index on ties: an
+      // entry moves down only for a strictly larger value) in one pass
+      float inv = 0.0f;
+      if (t < p.M) {
+        float m = -INFINITY;
+        float vl[KMAX];
+        int il[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          vl[j] = -INFINITY;
+          il[j] = -1;
+        }
+        for (int e = 0; e < E; ++e) {
+          const float l = s_lg[e * kRgLgStride + r];
+          m = fmaxf(m, l);
+          if (l > vl[KMAX - 1] || il[KMAX - 1] < 0) {
+            float cv = l;
+            int ci = e;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+              if (ci >= 0 && (il[j] < 0 || cv > vl[j])) {
+                const float tv = vl[j];
+                const int ti = il[j];
+                vl[j] = cv;
+                il[j] = ci;
+                cv = tv;
+                ci = ti;
+              }
+            }
+          }
+        }
+        float zsum = 0.0f;
+        for (int e = 0; e < E; ++e) {
+          const float z = expf(s_lg[e * kRgLgStride + r] - m);
+          s_lg[e * kRgLgStride + r] = z;
+          zsum += z;
+        }
+        inv = 1.0f / zsum;
+        float psum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < p.k) {
+            vl[j] = expf(vl[j] - m) * inv;
+            psum += vl[j];
+          }
+        const float denom = psum + 1e-20f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < p.k) {
+            p.topk_idx[static_cast<int64_t>(t) * p.k + j] = il[j];
+            p.topk_w[static_cast<int64_t>(t) * p.k + j] = vl[j] / denom;
+          }
+      }
+      __syncwarp();
+      if (p.probs != nullptr) {  // p = z / sum z, the warp's 32 rows, coalesced
+        for (int i = 0; i < 32; ++i) {
+          const int row = sub * 32 + i;
+          const float inv_i = __shfl_sync(0xffffffffu, inv, i);
+          if (m0 + row >= p.M) break;
+          for (int e = lane; e < E; e += 32)
+            p.probs[static_cast<int64_t>(m0 + row) * E + e] = s_lg[e * kRgLgStride + row] * inv_i;
+        }
+      }
+      tc_fence_before();
+    }
   }
 
   // ------------------------------------------------------------ tear-down

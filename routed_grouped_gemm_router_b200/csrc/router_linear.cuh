@@ -126,7 +126,7 @@ template <int KIND, int KMAX = 1>
 __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid_constant__ RouterGemmParams p) {
   constexpr bool kRoute = (KIND == kRgLogitsRoute);
   constexpr bool kAMN = (KIND == kRgWgrad);  // A = X^T: M (hidden) contiguous
-  constexpr bool kBMN = (KIND != kRgLogits); // B = dl3 (wgrad) or W3 (dgrad): N contiguous
+  constexpr bool kBMN = (KIND == kRgWgrad || KIND == kRgDgrad);  // B = dl3 (wgrad) or W3 (dgrad): N contiguous
   constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
   constexpr uint32_t kBLbo = kBMN ? 8192u : 16u;
   constexpr uint32_t kAStep = kAMN ? 2048u : 32u;  // bytes per 16-deep K step

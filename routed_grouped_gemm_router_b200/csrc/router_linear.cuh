@@ -448,10 +448,11 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
         }
       }
       // max and top-k (logit descending, lower expert index on ties: an
-      // entry moves down only for a strictly larger value) in one pass
+      // entry moves down only for a strictly larger value) in one pass, 8
+      // logits at a time with independent maxima; then z = exp(l - max) and
+      // its sum the same way (partial sums added in a fixed order)
       float inv = 0.0f;
       if (t < p.M) {
-        float m = -INFINITY;
         float vl[KMAX];
         int il[KMAX];
 #pragma unroll
@@ -459,31 +460,50 @@ __global__ void __launch_bounds__(kRgThreads, 1) router_gemm_kernel(const __grid
           vl[j] = -INFINITY;
           il[j] = -1;
         }
-        for (int e = 0; e < E; ++e) {
-          const float l = s_lg[e * kRgLgStride + r];
-          m = fmaxf(m, l);
-          if (l > vl[KMAX - 1] || il[KMAX - 1] < 0) {
-            float cv = l;
-            int ci = e;
+        float mx[8];
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-              if (ci >= 0 && (il[j] < 0 || cv > vl[j])) {
-                const float tv = vl[j];
-                const int ti = il[j];
-                vl[j] = cv;
-                il[j] = ci;
-                cv = tv;
-                ci = ti;
+        for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+        for (int e0 = 0; e0 < E; e0 += 8) {
+          float lv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) lv[u] = (e0 + u < E) ? s_lg[(e0 + u) * kRgLgStride + r] : -INFINITY;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], lv[u]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (e0 + u < E && (lv[u] > vl[KMAX - 1] || il[KMAX - 1] < 0)) {
+              float cv = lv[u];
+              int ci = e0 + u;
+#pragma unroll
+              for (int j = 0; j < KMAX; ++j) {
+                if (ci >= 0 && (il[j] < 0 || cv > vl[j])) {
+                  const float tv = vl[j];
+                  const int ti = il[j];
+                  vl[j] = cv;
+                  il[j] = ci;
+                  cv = tv;
+                  ci = ti;
+                }
               }
             }
           }
         }
-        float zsum = 0.0f;
-        for (int e = 0; e < E; ++e) {
-          const float z = expf(s_lg[e * kRgLgStride + r] - m);
-          s_lg[e * kRgLgStride + r] = z;
-          zsum += z;
+        const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        float zs[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) zs[u] = 0.0f;
+        for (int e0 = 0; e0 < E; e0 += 8) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (e0 + u < E) {
+              const float z = expf(s_lg[(e0 + u) * kRgLgStride + r] - m);
+              s_lg[(e0 + u) * kRgLgStride + r] = z;
+              zs[u] += z;
+            }
+          }
         }
+        const float zsum = ((zs[0] + zs[1]) + (zs[2] + zs[3])) + ((zs[4] + zs[5]) + (zs[6] + zs[7]));
         inv = 1.0f / zsum;
         float psum = 0.0f;
 #pragma unroll

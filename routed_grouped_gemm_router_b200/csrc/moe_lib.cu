@@ -330,8 +330,11 @@ int launch_router_gemm(const RouterGemmParams& p, cudaStream_t s, int slot) {
 }
 
 // Logits + routing in one launch (clusters of two CTAs per 128-token tile).
+// Off by default: measured slower than split-K logits + the routing kernel
+// (77 vs 48 us on T 8192, H 2048, E 128, k 8): the routing epilogue, one
+// thread per token over four warps, takes about 43 us.
 #ifndef MOE_ROUTER_FUSED_ROUTE
-#define MOE_ROUTER_FUSED_ROUTE 1
+#define MOE_ROUTER_FUSED_ROUTE 0
 #endif
 constexpr bool kRouterFusedRoute = MOE_ROUTER_FUSED_ROUTE != 0;
 template <int KMAX>

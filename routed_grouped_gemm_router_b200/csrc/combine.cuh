@@ -9,6 +9,12 @@
 #pragma once
 #include "common.cuh"
 
+// The expert outputs are read once: load them with the streaming hint
+// (evict-first) so they do not displace reused data from L2.
+#ifndef MOE_COMBINE_STREAM_LOADS
+#define MOE_COMBINE_STREAM_LOADS 1
+#endif
+
 namespace moe {
 
 template <int KMAX>
@@ -32,8 +38,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       uint4 v[KMAX];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
+      for (int j = 0; j < KMAX; ++j) {
+#if MOE_COMBINE_STREAM_LOADS
+        v[j] = (rows[j] >= 0) ? __ldcs(O + rows[j] * vec_per_row + c) : make_uint4(0, 0, 0, 0);
+#else
         v[j] = (rows[j] >= 0) ? __ldg(O + rows[j] * vec_per_row + c) : make_uint4(0, 0, 0, 0);
+#endif
+      }
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         if (rows[j] >= 0) {

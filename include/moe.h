@@ -27,12 +27,7 @@
  *    index tensors are int32; weights/logits/gradients of the router are fp32.
  *  - Streams: each call only enqueues work on `stream` (NULL = legacy default
  *    stream) and returns without synchronising. Nothing is read back to the
- *    host; the per-expert counts never leave the device. moe_layer_bwd also
- *    runs two memory-bound kernels on an internal stream of the device,
- *    forked from `stream` and joined back to it with events before it
- *    returns, so every result is ordered on `stream` as usual; that stream
- *    and its events are created by the device's first moe_layer_bwd call
- *    (make that call before capturing a graph of it).
+ *    host; the per-expert counts never leave the device.
  *  - Errors: arguments are checked before anything is launched. A bad shape,
  *    a NULL required pointer or a pointer that is not 16-byte aligned returns
  *    MOE_ERR_INVALID_ARG, a workspace that is too small MOE_ERR_WORKSPACE, a

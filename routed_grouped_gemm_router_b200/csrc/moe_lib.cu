@@ -81,35 +81,6 @@ int current_device_info(DeviceInfo** out) {
   return d.supported ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
-// A second stream per device on which moe_layer_bwd runs the memory-bound
-// kernels that do not feed the weight-gradient GEMMs (routing-logit gradient,
-// dX combine), so they overlap those GEMMs; forked from and joined back to
-// the caller's stream with events. Created on the device's first backward.
-struct SideStream {
-  int ready = 0;
-  cudaStream_t s = nullptr;
-  cudaEvent_t ev_dgrad_down = nullptr, ev_dgrad_gate_up = nullptr, ev_done = nullptr;
-  std::mutex mu;  // one call at a time enqueues on the side stream
-};
-SideStream g_side[kMaxDevices];
-
-int side_stream(SideStream** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  SideStream& ss = g_side[dev];
-  std::lock_guard<std::mutex> lock(g_dev_mu);
-  if (!ss.ready) {
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.ev_dgrad_down, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.ev_dgrad_gate_up, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.ev_done, cudaEventDisableTiming) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    ss.ready = 1;
-  }
-  *out = &ss;
-  return MOE_OK;
-}
-
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
 // library does not link libcuda directly.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -669,20 +640,6 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
       return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  SideStream* side = nullptr;
-  if (int st = side_stream(&side)) return st;
-  std::lock_guard<std::mutex> side_lock(side->mu);
-  // once forked, the side stream is joined back to the caller's stream on
-  // every return path
-  bool forked = false;
-  struct Join {
-    SideStream* ss;
-    cudaStream_t main;
-    const bool& forked;
-    ~Join() {
-      if (forked && cudaEventRecord(ss->ev_done, ss->s) == cudaSuccess) cudaStreamWaitEvent(main, ss->ev_done, 0);
-    }
-  } join{side, stream, forked};
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   moe_bf16* dYp = reinterpret_cast<moe_bf16*>(w8 + L.dYp);
   moe_bf16* dGU = reinterpret_cast<moe_bf16*>(w8 + L.dGU);
@@ -754,21 +711,6 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
                         : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown))
       return st;
   }
-  // 3b. routing-logit gradient (needs only the dgrad-down's partial dw),
-  //     on the side stream
-  if (cudaEventRecord(side->ev_dgrad_down, stream) != cudaSuccess ||
-      cudaStreamWaitEvent(side->s, side->ev_dgrad_down, 0) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  forked = true;
-  {
-    ProfScope ps(kProfRouterBwd, side->s);
-    int blocks = (T + 7) / 8;
-    if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
-    if (launch_pdl(router_bwd_kernel, dim3(blocks), dim3(256), sizeof(float) * 8 * E, side->s, probs, topk_idx,
-                   topk_w, static_cast<const float*>(dw_part), pair_pos, kDwSlotsPerNTile * nt_dgrad_down,
-                   static_cast<int64_t>(T), E, k, dlogits) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
   {
     GemmParams bx = base_params(E, P, offsets);
@@ -786,14 +728,10 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
                                               kProfDgradGateUp))
       return st;
   }
-  // 5. dX[t] = sum_j dXp[pair_pos[t*k+j]], on the side stream, overlapping
-  //    the weight-gradient GEMMs (which read neither dXp nor dX)
-  if (cudaEventRecord(side->ev_dgrad_gate_up, stream) != cudaSuccess ||
-      cudaStreamWaitEvent(side->s, side->ev_dgrad_gate_up, 0) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  // 5. dX[t] = sum_j dXp[pair_pos[t*k+j]]
   {
-    ProfScope ps(kProfCombineDx, side->s);
-    if (launch_combine(dXp, pair_pos, T, k, H, dX, side->s, dev->num_sms) != cudaSuccess) return MOE_ERR_CUDA;
+    ProfScope ps(kProfCombineDx, stream);
+    if (launch_combine(dXp, pair_pos, T, k, H, dX, stream, dev->num_sms) != cudaSuccess) return MOE_ERR_CUDA;
   }
   // 6. weight gradients, K = the expert's rows. Each launch first writes
   //    per-expert copies of its two tensor maps, clipped at the segment end.
@@ -851,6 +789,16 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     if (int st = gather ? launch_gemm<kBwdWgrad, kGatherA>(wd, grid, stream, kProfWgradDown)
                         : launch_gemm<kBwdWgrad>(wd, grid, stream, kProfWgradDown))
       return st;
+  }
+  // 7. router logits gradient
+  {
+    ProfScope ps(kProfRouterBwd, stream);
+    int blocks = (T + 7) / 8;
+    if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
+    if (launch_pdl(router_bwd_kernel, dim3(blocks), dim3(256), sizeof(float) * 8 * E, stream, probs, topk_idx, topk_w,
+                   static_cast<const float*>(dw_part), pair_pos, kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k,
+                   dlogits) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }

@@ -11,15 +11,20 @@
 //    even CTA issues the MMA for both, and each CTA's TMEM receives its 128
 //    accumulator rows. Per CTA a 64-deep K step is 32 KiB, so a 6-deep
 //    TMA ring fits in shared memory;
-//  * 10 warps per CTA: warp 0 issues TMA loads (and L2 prefetches ahead of
-//    them), warp 1 issues MMAs (even CTA) and owns the TMEM allocation,
+//  * 10 warps per CTA: warp 0 issues TMA loads, warp 1 issues MMAs (even
+//    CTA) and owns the TMEM allocation,
 //    warps 2-9 run the epilogue, two per TMEM sub-partition;
 //  * both CTAs' loads complete on the even CTA's "full" mbarrier; the MMA
 //    warp's commits release the "empty" barriers of both CTAs; the fp32
 //    accumulator is double-buffered in TMEM (2 x 256 columns) so the
 //    epilogue of tile i overlaps the main loop of tile i+1;
 //  * the tile list is built on the device from the per-expert offsets, so the
-//    host never learns the counts and experts without rows cost nothing.
+//    host never learns the counts and experts without rows cost nothing;
+//  * segment tails of 1..128 rows run in a second, one-CTA instance of the
+//    kernel (CG = 1: 128 x 256 x 16 MMAs, each CTA staging all 256 B rows)
+//    that is launched first on a few whole TPCs; the pair instance, launched
+//    right after on the other SMs, runs concurrently with it (a 256-row pair
+//    tile would spend at least half its tensor work on padding rows there).
 //
 // Variants (all D = A * B^T with bf16 operands and fp32 accumulation):
 //  FwdGateUp   A = Xp[P,H] (K-major), B = gate rows (even CTA) and up rows
@@ -53,23 +58,39 @@ constexpr int kBN = 256;        // columns of a tile (accumulator columns per CT
 constexpr int kBNc = 128;       // B rows (N) staged per CTA
 constexpr int kBK = 64;
 constexpr int kUmmaK = 16;
-constexpr int kStages = 6;
+constexpr int kStages = 6;                   // ring depth of the pair instance
 constexpr int kATileBytes = kBMc * kBK * 2;  // 16 KiB
-constexpr int kBTileBytes = kBNc * kBK * 2;  // 16 KiB
+constexpr int kBTileBytes = kBNc * kBK * 2;  // 16 KiB per CTA of a pair
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
+// Per CTA-group constants: ring depth, bytes of B staged per CTA.
+template <int CG> struct CgCfg {
+  static constexpr int kStages = CG == 2 ? 6 : 4;
+  static constexpr int kBBytes = CG == 2 ? kBTileBytes : 2 * kBTileBytes;
+  static constexpr int kStageBytes = kATileBytes + kBBytes;
+};
+// Segment tails of 1..128 rows run as one-CTA tiles (0: every row-grouped
+// tile is a pair tile).
+#ifndef MOE_TAIL_TILES
+#define MOE_TAIL_TILES 1
+#endif
+constexpr bool kTailTiles = MOE_TAIL_TILES != 0;
+
+// Row tiles of a segment of `rows` rows handled by the CG instance (tails
+// split off only when `tails` is set).
+template <int CG>
+__host__ __device__ __forceinline__ int seg_row_tiles(int rows, bool tails) {
+  if (!tails) return CG == 2 ? (rows + 255) / 256 : 0;
+  const int full = rows / 256, tail = rows - 256 * (rows / 256);
+  return CG == 2 ? full + (tail > 128 ? 1 : 0) : (tail > 0 && tail <= 128 ? 1 : 0);
+}
 // Epilogue warps: 4 (one per TMEM sub-partition) or 8 (two per sub-partition,
 // each half of the columns).
 #ifndef MOE_EPI_WARPS
 #define MOE_EPI_WARPS 8
 #endif
-// K blocks the L2 prefetch cursor runs ahead of the TMA loads (0: off).
-#ifndef MOE_PREFETCH_AHEAD
-#define MOE_PREFETCH_AHEAD 0
-#endif
 constexpr int kEpiWarps = MOE_EPI_WARPS;
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "4 or 8 epilogue warps");
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
-constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
 // Epilogue outputs are written with the streaming hint (evict-first in L2)
 // so they do not push reused operand tiles out of L2.
 #ifndef MOE_STREAM_STORES
@@ -83,7 +104,7 @@ constexpr int kPrefetchAhead = MOE_PREFETCH_AHEAD;
 #endif
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kMaxExperts = 1024;
-constexpr int kNumBarriers = 2 * kStages + 5;
+constexpr int kNumBarriers = 2 * kStages + 5;  // sized for the deeper (pair) ring
 // Epilogue staging: per epilogue warp 32 rows x 32 bf16 (64 bytes per row).
 // The four 16-byte pieces of row r are stored at piece (m ^ ((r >> 1) & 3)),
 // which keeps both the row-wise writes (8 rows per quarter-warp phase) and
@@ -121,10 +142,14 @@ struct GemmParams {
   int gather_k;               // pair id -> token: q / gather_k
   int gather_rows;
   int gather_cols;
+  int tails;                  // row-grouped kinds: segment tails of 1..128 rows go to the one-CTA instance
+  int wait_at_end;            // pair instance launched after a one-CTA instance: wait for it at the end
 };
 
+template <int CG>
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
-  return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes + kNumBarriers * 8 + 16 +
+  return 1024 /*alignment slack*/ + static_cast<size_t>(CgCfg<CG>::kStages) * CgCfg<CG>::kStageBytes +
+         kNumBarriers * 8 + 16 +
          2 * static_cast<size_t>(E + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * kStageWarpBytes;
 }
 
@@ -135,7 +160,7 @@ struct TileInfo {
   int num_kb;   // K blocks
 };
 
-template <int KIND>
+template <int KIND, int CG>
 __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
                                                 const int* s_tstart) {
   TileInfo ti;
@@ -157,14 +182,15 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.e = lo;
     const int local = t - s_tstart[lo];
 #if MOE_TILE_M_FASTEST
-    const int m_tiles_e = (s_off[lo + 1] - s_off[lo] + kBM - 1) / kBM;
+    const int m_tiles_e = seg_row_tiles<CG>(s_off[lo + 1] - s_off[lo], p.tails != 0);
     ti.n_blk = local / m_tiles_e;
     ti.m_blk = local - ti.n_blk * m_tiles_e;
 #else
     ti.m_blk = local / p.n_tiles;
     ti.n_blk = local - ti.m_blk * p.n_tiles;
 #endif
-    ti.row0 = s_off[lo] + ti.m_blk * kBM;
+    // pair tiles start at 256-row steps; the one-CTA tile is the segment's tail
+    ti.row0 = s_off[lo] + (CG == 2 ? ti.m_blk * kBM : ((s_off[lo + 1] - s_off[lo]) / kBM) * kBM);
     ti.rows = s_off[lo + 1] - ti.row0;
     ti.num_kb = (p.K + kBK - 1) / kBK;
   }
@@ -267,13 +293,18 @@ __device__ __forceinline__ void dgrad_down_load(const GemmParams& p, int64_t wro
 __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
-template <int KIND, int GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+// CG = 2: CTA pairs (launched as clusters of two); CG = 1: one CTA per tile,
+// the segment tails of 1..128 rows (row-grouped kinds without gathering;
+// launched as clusters of two as well, so the pair instance gets whole TPCs).
+template <int KIND, int GATHER, int CG = 2>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool kWgrad = (KIND == kBwdWgrad);
+  static_assert(CG == 2 || (!kWgrad && GATHER == kNoGather), "one-CTA tiles: row-grouped kinds, no gathering");
+  using Cfg = CgCfg<CG>;
+  constexpr int kSt = Cfg::kStages;
   constexpr bool kAMN = kWgrad;
   constexpr bool kBMN = (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || kWgrad);
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, kAMN, kBMN);
+  constexpr uint32_t kIdesc = idesc_bf16_f32(CG == 2 ? kBM : kBMc, kBN, kAMN, kBMN);
   constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
   constexpr uint32_t kBLbo = kBMN ? 8192u : 16u;
   constexpr uint32_t kAStep = kAMN ? 2048u : 32u;  // bytes per UMMA_K step
@@ -282,8 +313,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kATileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* sB = smem + kSt * kATileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSt * Cfg::kStageBytes);
   uint64_t* full_bar = bars;                 // even CTA: both CTAs' TMA bytes of a stage
   uint64_t* empty_bar = bars + kStages;      // each CTA: its stage may be refilled
   uint64_t* tfull_bar = bars + 2 * kStages;  // each CTA: accumulator buffer ready
@@ -297,19 +328,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
-  const int pair = blockIdx.x >> 1;
-  const int num_pairs = gridDim.x >> 1;
+  // CG = 2: 0 = even CTA (issues the MMAs), 1 = odd CTA; CG = 1: always 0
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int pair = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int num_pairs = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 2 * kEpiWarps);  // one arrival per epilogue warp of the pair
+      mbar_init(&tempty_bar[a], CG * kEpiWarps);  // one arrival per epilogue warp of the pair / CTA
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -321,12 +353,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if constexpr (GATHER != kNoGather) tma_prefetch_desc(&p.tmG);
   }
   if (warp == 1) {
-    tmem_alloc_pair(s_tmem, kTmemCols);
-    tmem_relinquish_pair();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(s_tmem, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, kTmemCols);
+      tmem_relinquish();
+    }
   }
-  // everything above touches no global memory; from here on this kernel reads
-  // its predecessors' results
-  griddep_wait();
+  // Everything above touches no global memory; from here on this kernel
+  // reads its predecessors' results, so it waits for them first. A pair
+  // instance launched right after a one-CTA instance (wait_at_end) starts
+  // only once every one-CTA CTA has passed this wait, so its inputs are
+  // complete already: it runs concurrently with the one-CTA instance and
+  // waits for it at its end instead, so the next kernel sees both.
+  if (!(CG == 2 && p.wait_at_end)) griddep_wait();
   griddep_launch_dependents();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
   __syncthreads();
@@ -337,7 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int local = 0;
     for (int i = 0; i < per; ++i) {
       const int e = e0 + i;
-      if (e < p.E) local += ((s_off[e + 1] - s_off[e] + kBM - 1) / kBM) * p.n_tiles;
+      if (e < p.E) local += seg_row_tiles<CG>(s_off[e + 1] - s_off[e], p.tails != 0) * p.n_tiles;
     }
     const int incl = warp_inclusive_scan(local);
     int run = incl - local;
@@ -345,26 +386,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int e = e0 + i;
       if (e < p.E) {
         s_tstart[e] = run;
-        run += ((s_off[e + 1] - s_off[e] + kBM - 1) / kBM) * p.n_tiles;
+        run += seg_row_tiles<CG>(s_off[e + 1] - s_off[e], p.tails != 0) * p.n_tiles;
       }
     }
     if (lane == 31) s_tstart[p.E] = incl;
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
+  if constexpr (CG == 2) cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int total_tiles = kWgrad ? p.E * p.m_tiles * p.n_tiles : s_tstart[p.E];
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
-    // Loads K block kb of tile ti (this CTA's A half and B half) into a ring
-    // stage, or with prefetch_only just asks TMA to bring the same boxes into
-    // L2. A prefetch cursor runs kPrefetchAhead K blocks (across tile
-    // boundaries) ahead of the loads so first touches of weight and
-    // activation tiles start their DRAM reads early.
-    auto issue = [&](const TileInfo& ti, int kb, bool prefetch_only, uint8_t* a_dst, uint8_t* b_dst, uint32_t fb) {
+    // Loads K block kb of tile ti (this CTA's A rows and its share of B: half
+    // of the 256 B rows in a pair, all of them in a one-CTA tile) into a
+    // ring stage. In a pair both CTAs' bytes complete on the even CTA's full
+    // barrier (a cluster address); a one-CTA tile uses its own. A gathered
+    // operand (GATHER) is not loaded here but by the gathering producer below.
+    auto issue = [&](const TileInfo& ti, int kb, bool prefetch_only, uint8_t* a_dst, uint8_t* b_dst, uint32_t fb,
+                     uint64_t* fb_local) {
+      (void)prefetch_only;
       const CUtensorMap* mapA = &p.tmA;
       const CUtensorMap* mapB = &p.tmB;
       if constexpr (kWgrad) {
@@ -372,34 +415,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         mapB = p.expert_maps + p.E + ti.e;
       }
       const int kx = kb * kBK;
-      int ax, ay, bx, by, nbox_a = 1, nbox_b = 1;
+      const int r = static_cast<int>(rank);
+      // box c of B lands 8 KiB (MN-major boxes of 64 x 64) or 16 KiB
+      // (K-major boxes of 128 rows) after the previous one
+      int ax, ay, bx, by, nbox_a = 1, nbox_b = 1, b_step_x = 0, b_step_y = 0, b_step_bytes = 0;
       if constexpr (KIND == kFwdGateUp) {
-        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
-        // even CTA: the tile's 128 gate rows; odd CTA: the matching up rows
-        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBNc + static_cast<int>(rank) * p.I;
+        ax = kx; ay = ti.row0 + r * kBMc;
+        // gate rows of the N block (even CTA / first box), then the matching up rows
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBNc + r * p.I;
+        if constexpr (CG == 1) { nbox_b = 2; b_step_y = p.I; b_step_bytes = kBTileBytes; }
       } else if constexpr (KIND == kFwdDown) {
-        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
-        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBN + static_cast<int>(rank) * kBNc;
+        ax = kx; ay = ti.row0 + r * kBMc;
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBN + r * kBNc;
+        if constexpr (CG == 1) { nbox_b = 2; b_step_y = kBNc; b_step_bytes = kBTileBytes; }
       } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
-        ax = kx; ay = ti.row0 + static_cast<int>(rank) * kBMc;
-        bx = ti.n_blk * kBN + static_cast<int>(rank) * kBNc; by = ti.e * p.b_rows + kx;
-        nbox_b = 2;
+        ax = kx; ay = ti.row0 + r * kBMc;
+        bx = ti.n_blk * kBN + r * kBNc; by = ti.e * p.b_rows + kx;
+        nbox_b = CG == 2 ? 2 : 4; b_step_x = 64; b_step_bytes = 8192;
       } else {  // wgrad: K rows are the expert's permuted rows
-        ax = ti.m_blk * kBM + static_cast<int>(rank) * kBMc; ay = ti.row0 + kx;
-        bx = ti.n_blk * kBN + static_cast<int>(rank) * kBNc; by = ay;
+        ax = ti.m_blk * kBM + r * kBMc; ay = ti.row0 + kx;
+        bx = ti.n_blk * kBN + r * kBNc; by = ay;
         nbox_a = 2;
-        nbox_b = 2;
+        nbox_b = 2; b_step_x = 64; b_step_bytes = 8192;
       }
       if constexpr (GATHER != kGatherA) {
         for (int c = 0; c < nbox_a; ++c) {
-          if (prefetch_only) tma_prefetch_2d(mapA, ax + 64 * c, ay);
-          else tma_load_2d_pair(a_dst + 8192 * c, mapA, fb, ax + 64 * c, ay);
+          if constexpr (CG == 2) tma_load_2d_pair(a_dst + 8192 * c, mapA, fb, ax + 64 * c, ay);
+          else tma_load_2d(a_dst + 8192 * c, mapA, fb_local, ax + 64 * c, ay);
         }
       }
       if constexpr (GATHER != kGatherB) {
         for (int c = 0; c < nbox_b; ++c) {
-          if (prefetch_only) tma_prefetch_2d(mapB, bx + 64 * c, by);
-          else tma_load_2d_pair(b_dst + 8192 * c, mapB, fb, bx + 64 * c, by);
+          if constexpr (CG == 2)
+            tma_load_2d_pair(b_dst + b_step_bytes * c, mapB, fb, bx + b_step_x * c, by + b_step_y * c);
+          else
+            tma_load_2d(b_dst + b_step_bytes * c, mapB, fb_local, bx + b_step_x * c, by + b_step_y * c);
         }
       }
     };
@@ -407,46 +457,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      // prefetch cursor: tile pf_t, K block pf_kb; pf_lead = blocks ahead of the loads
-      int pf_t = pair, pf_kb = 0, pf_lead = 0;
-      TileInfo pf_ti;
-      if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
       for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
-        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        const TileInfo ti = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
         if constexpr (kWgrad) {
           if (ti.num_kb == 0) continue;
           tensormap_acquire(p.expert_maps + ti.e);
           tensormap_acquire(p.expert_maps + p.E + ti.e);
         }
         for (int kb = 0; kb < ti.num_kb; ++kb) {
-          while (pf_lead < kPrefetchAhead && pf_t < total_tiles) {
-            if (pf_kb < pf_ti.num_kb) {
-              if constexpr (kWgrad) {
-                if (pf_kb == 0) {
-                  tensormap_acquire(p.expert_maps + pf_ti.e);
-                  tensormap_acquire(p.expert_maps + p.E + pf_ti.e);
-                }
-              }
-              issue(pf_ti, pf_kb, true, nullptr, nullptr, 0);
-              ++pf_kb;
-              ++pf_lead;
-            } else {
-              pf_t += num_pairs;
-              pf_kb = 0;
-              if (pf_t < total_tiles) pf_ti = decode_tile<KIND>(pf_t, p, s_off, s_tstart);
-            }
-          }
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
             report(MOE_ERR_TIMEOUT);
             *s_abort = 1;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
-          issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes,
-                mapa_shared(smem_u32(&full_bar[stage]), 0));
-          if (pf_lead > 0) --pf_lead;
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], CG * Cfg::kStageBytes);
+          issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * Cfg::kBBytes,
+                CG == 2 ? mapa_shared(smem_u32(&full_bar[stage]), 0) : 0u, &full_bar[stage]);
           ++issued;
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1u;
           }
@@ -456,10 +484,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // last phases there means no load of the pair is still in flight when
       // the pair leaves (immediate in normal operation).
       if (rank == 0) {
-        const int inflight = issued < kStages ? issued : kStages;
+        const int inflight = issued < kSt ? issued : kSt;
         for (int i = 0; i < inflight; ++i) {
           if (--stage < 0) {
-            stage = kStages - 1;
+            stage = kSt - 1;
             phase ^= 1u;
           }
           mbar_wait(&full_bar[stage], phase);
@@ -491,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         return t < 0 ? 0 : (t >= p.gather_rows ? p.gather_rows - 1 : t);
       };
       auto tile_pairs = [&](int t, int32_t (&q)[4]) {
-        const TileInfo tn = decode_tile<KIND>(t, p, s_off, s_tstart);
+        const TileInfo tn = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int r = static_cast<int>(rank) * kBMc + 4 * lane + m;
@@ -505,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (pair < total_tiles && !*s_abort) tile_pairs(pair, q_nxt);
       }
       for (int t = pair; t < total_tiles && !__any_sync(0xffffffffu, *s_abort != 0); t += num_pairs) {
-        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        const TileInfo ti = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
         if constexpr (kWgrad) {
           if (ti.num_kb == 0) continue;
           if (lane == 0) {
@@ -550,7 +578,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (lane == 0) {
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
-            issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes, fb);
+            issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * kBTileBytes, fb, &full_bar[stage]);
           }
           uint8_t* g_tile = (GATHER == kGatherA) ? sA + stage * kATileBytes : sB + stage * kBTileBytes;
           int gx = kb * kBK, goff = 512 * lane;
@@ -585,13 +613,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer (even CTA)
     if (rank == 0) {
-      const uint32_t peer_empty0 = mapa_shared(smem_u32(&empty_bar[0]), 1);
-      const uint32_t peer_tfull0 = mapa_shared(smem_u32(&tfull_bar[0]), 1);
+      const uint32_t peer_empty0 = CG == 2 ? mapa_shared(smem_u32(&empty_bar[0]), 1) : 0u;
+      const uint32_t peer_tfull0 = CG == 2 ? mapa_shared(smem_u32(&tfull_bar[0]), 1) : 0u;
       int stage = 0;
       uint32_t phase = 0;
       int tcount = 0;
       for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
-        const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+        const TileInfo ti = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
         if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogues write zeros
         const int acc = tcount & 1;
         if (!warp_wait(&tempty_bar[acc], ((tcount >> 1) & 1) ^ 1u)) {
@@ -610,18 +638,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           if (lane == 0) {
             const uint32_t a_addr = smem_u32(sA + stage * kATileBytes);
-            const uint32_t b_addr = smem_u32(sB + stage * kBTileBytes);
+            const uint32_t b_addr = smem_u32(sB + stage * Cfg::kBBytes);
 #pragma unroll
             for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
               const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
               const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
-              umma_bf16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              if constexpr (CG == 2) umma_bf16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              else umma_bf16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
             }
-            umma_commit_pair(smem_u32(&empty_bar[stage]));
-            umma_commit_pair(peer_empty0 + stage * 8);
+            if constexpr (CG == 2) {
+              umma_commit_pair(smem_u32(&empty_bar[stage]));
+              umma_commit_pair(peer_empty0 + stage * 8);
+            } else {
+              umma_commit(&empty_bar[stage]);
+            }
           }
           __syncwarp();
-          if (++stage == kStages) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1u;
           }
@@ -632,14 +665,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         if (lane == 0) {
-          umma_commit_pair(smem_u32(&tfull_bar[acc]));
-          umma_commit_pair(peer_tfull0 + acc * 8);
+          if constexpr (CG == 2) {
+            umma_commit_pair(smem_u32(&tfull_bar[acc]));
+            umma_commit_pair(peer_tfull0 + acc * 8);
+          } else {
+            umma_commit(&tfull_bar[acc]);
+          }
         }
         __syncwarp();
         ++tcount;
       }
       // all MMAs of the pair must finish before TMEM is released
-      if (lane == 0) umma_commit_pair(smem_u32(drain_bar));
+      if (lane == 0) {
+        if constexpr (CG == 2) umma_commit_pair(smem_u32(drain_bar));
+        else umma_commit(drain_bar);
+      }
       __syncwarp();
       warp_wait(drain_bar, 0);
     }
@@ -657,11 +697,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int tr_row = lane >> 2;  // transposed domain: row 8*i + tr_row
     const int tr_q = lane & 3;     // transposed domain: columns 8*tr_q..+7 of the chunk
     uint8_t* stg = s_stage + (warp - 2) * kStageWarpBytes;
-    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t leader_tempty0 = CG == 2 ? mapa_shared(smem_u32(&tempty_bar[0]), 0) : 0u;
     constexpr int kChunks = (KIND == kFwdGateUp ? 128 : kBN) / 32 / (kEpiWarps / 4);  // chunks per warp
     int tcount = 0;
     for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
-      const TileInfo ti = decode_tile<KIND>(t, p, s_off, s_tstart);
+      const TileInfo ti = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
       // this CTA's 128 rows of the pair tile, this warp's 32 of them
       const int cta_row0 = static_cast<int>(rank) * kBMc + sub * 32;
       const int tile_rows = kWgrad ? p.M - ti.m_blk * kBM : ti.rows;
@@ -829,7 +869,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #define MOE_TEMPTY_RELAXED 1
 #endif
       if (lane == 0) {
-        if (MOE_TEMPTY_RELAXED) mbar_arrive_cluster_relaxed(leader_tempty0 + acc * 8);
+        if constexpr (CG == 1) mbar_arrive(&tempty_bar[acc]);
+        else if (MOE_TEMPTY_RELAXED) mbar_arrive_cluster_relaxed(leader_tempty0 + acc * 8);
         else mbar_arrive_cluster(leader_tempty0 + acc * 8);
       }
       ++tcount;
@@ -839,11 +880,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // ------------------------------------------------------------- tear-down
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // the pair's MMAs, loads and TMEM reads are all finished
+  if constexpr (CG == 2) cluster_sync_all();  // the pair's MMAs, loads and TMEM reads are all finished
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
+  // a pair instance that did not wait at its start completes only after the
+  // one-CTA instance launched before it
+  if (CG == 2 && p.wait_at_end) griddep_wait();
 }
 
 // Writes, for each expert e, copies of the A and B tensor maps of the weight

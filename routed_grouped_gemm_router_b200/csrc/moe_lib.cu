@@ -197,16 +197,41 @@ struct ProfScope {
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-template <int KIND, int GATHER = kNoGather>
-int launch_gemm(const GemmParams& p, int grid, cudaStream_t s, int slot) {
-  const size_t smem = gemm_smem_bytes(p.E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int KIND, int GATHER, int CG>
+int launch_gemm_instance(const GemmParams& p, int grid, cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes<CG>(p.E);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND, GATHER, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  ProfScope ps(slot, s);
-  if (launch_pdl(grouped_gemm_kernel<KIND, GATHER>, dim3(grid), dim3(kGemmThreads), smem, s, p) != cudaSuccess)
+  // both instances run as clusters of two, so each takes whole TPCs
+  if (launch_pdl_clustered(grouped_gemm_kernel<KIND, GATHER, CG>, dim3(grid), dim3(kGemmThreads), smem, s, 2u, p) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_status();
+}
+
+// One grouped GEMM. Row-grouped kinds without gathering with tail_ctas > 0:
+// the one-CTA instance over the segment tails of 1..128 rows on tail_ctas
+// CTAs, then the pair instance over the rest on the other SMs, concurrently
+// (grid is the pair instance's grid without tails). Otherwise the pair
+// instance alone over every tile.
+template <int KIND, int GATHER = kNoGather>
+int launch_gemm(GemmParams p, int grid, cudaStream_t s, int slot, int tail_ctas = 0, int num_sms = 0) {
+  ProfScope ps(slot, s);
+  if constexpr (KIND != kBwdWgrad && GATHER == kNoGather) {
+    if (kTailTiles && tail_ctas > 0) {
+      p.tails = 1;
+      p.wait_at_end = 0;
+      if (int st = launch_gemm_instance<KIND, GATHER, 1>(p, tail_ctas, s)) return st;
+      p.wait_at_end = 1;
+      int pg = num_sms - tail_ctas;
+      pg = (pg < grid ? pg : grid) & ~1;
+      return launch_gemm_instance<KIND, GATHER, 2>(p, pg > 2 ? pg : 2, s);
+    }
+  }
+  p.tails = 0;
+  p.wait_at_end = 0;
+  return launch_gemm_instance<KIND, GATHER, 2>(p, grid, s);
 }
 
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -220,6 +245,24 @@ inline int pair_grid(int64_t tiles, int num_sms) {
 }
 inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
   return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
+}
+// CTAs (even) for the one-CTA tail instance, from the expected work split:
+// about half the experts end in a tail of 1..128 rows (one CTA for one tile
+// time each), the full tiles cost two CTAs each (P / 256 of them). When the
+// average segment is 128 rows or less nearly every tile is a tail.
+inline int tail_ctas(int64_t P, int E, int num_sms) {
+  if (!kTailTiles || P == 0) return 0;
+  int c;
+  if (P <= static_cast<int64_t>(128) * E) {
+    c = num_sms - 4;
+  } else {
+    const double tail = 0.5 * E, full = 2.0 * static_cast<double>(P) / kBM;
+    c = static_cast<int>(num_sms * tail / (tail + full) + 0.5);
+  }
+  c &= ~1;
+  if (c < 2) c = 2;
+  if (c > num_sms - 4) c = (num_sms - 4) & ~1;
+  return c;
 }
 
 // The gathered operand of a GEMM: token-order rows [T, H] picked by
@@ -552,7 +595,7 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   gu.gu = gu_save;
   const int gu_grid = rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms);
   if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(gu, gu_grid, stream, kProfFwdGateUp)
-                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp))
+                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
     return st;
 
   GemmParams dn = base_params(E, P, offsets);
@@ -567,7 +610,7 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   dn.n_tiles = cdiv(H, kBN);
   dn.out = O;
   dn.out_ld = H;
-  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown);
+  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown, tail_ctas(P, E, dev->num_sms), dev->num_sms);
 }
 }  // namespace
 }  // namespace moe
@@ -680,7 +723,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     rc.gu = gu_ws;
     const int grid = rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms);
     if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(rc, grid, stream, kProfRecomputeGateUp)
-                        : launch_gemm<kFwdGateUp>(rc, grid, stream, kProfRecomputeGateUp))
+                        : launch_gemm<kFwdGateUp>(rc, grid, stream, kProfRecomputeGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
     gu = gu_ws;
   }
@@ -708,7 +751,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     bd.dw_part = dw_part;
     const int grid = rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms);
     if (int st = gather ? launch_gemm<kBwdDgradDown, kGatherA>(bd, grid, stream, kProfDgradDown)
-                        : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown))
+                        : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
   }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
@@ -725,7 +768,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     bx.out = dXp;
     bx.out_ld = H;
     if (int st = launch_gemm<kBwdDgradGateUp>(bx, rowgrouped_grid(P, E, bx.n_tiles, dev->num_sms), stream,
-                                              kProfDgradGateUp))
+                                              kProfDgradGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
   }
   // 5. dX[t] = sum_j dXp[pair_pos[t*k+j]]

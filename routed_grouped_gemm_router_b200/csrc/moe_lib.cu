@@ -247,16 +247,18 @@ inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
   return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
 }
 // CTAs (even) for the one-CTA tail instance, from the expected work split:
-// about half the experts end in a tail of 1..128 rows (one CTA for one tile
-// time each), the full tiles cost two CTAs each (P / 256 of them). When the
-// average segment is 128 rows or less nearly every tile is a tail.
+// about 0.65 E segments end in a tail of 1..128 rows (half of them for
+// evenly spread routing, more when a few experts take most rows and the
+// rest are small), one CTA for one tile time each; the full tiles cost two
+// CTAs each (P / 256 of them). When the average segment is 128 rows or less
+// nearly every tile is a tail.
 inline int tail_ctas(int64_t P, int E, int num_sms) {
   if (!kTailTiles || P == 0) return 0;
   int c;
   if (P <= static_cast<int64_t>(128) * E) {
     c = num_sms - 4;
   } else {
-    const double tail = 0.5 * E, full = 2.0 * static_cast<double>(P) / kBM;
+    const double tail = 0.65 * E, full = 2.0 * static_cast<double>(P) / kBM;
     c = static_cast<int>(num_sms * tail / (tail + full) + 0.5);
   }
   c &= ~1;

@@ -157,13 +157,19 @@ class ClockSampler:
 
     def _run(self):
         nv = self.nvml
+        mx = None
+        n = 0
+        pw = 0.0
         while not self.stop_flag:
             if self.active and nv is not None:
                 try:
+                    if mx is None:  # static: read once
+                        mx = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
                     sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
-                    mx = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
-                    pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
                     rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    if n % 4 == 0:  # power is an averaged reading: every 4th sample
+                        pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                    n += 1
                     self.rows.append((sm, mx, pw, rs))
                 except Exception:
                     pass

@@ -288,6 +288,7 @@ def workload_config(wl, args):
                         + (" + router Linear (fp32, on the GPU)" if getattr(args, "router_linear", False) else ""),
             "router_linear": bool(getattr(args, "router_linear", False)),
             "gather_fused": bool(getattr(args, "gather_fused", False)),
+            "cuda_graph": bool(getattr(args, "cuda_graph", False)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -300,6 +301,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qwen3-30b-a3b", choices=sorted(WORKLOADS))
     ap.add_argument("--forward-only", action="store_true")
+    ap.add_argument("--cuda-graph", action="store_true",
+                    help="capture one whole step in a CUDA graph after warm-up and time its replays")
     ap.add_argument("--gather-fused", action="store_true",
                     help="GEMMs read X / dY rows by token (no Xp / dYp copies) instead of the permuted copies")
     ap.add_argument("--router-linear", action="store_true",
@@ -371,10 +374,27 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
 
+    graph = None
+    if args.cuda_graph:
+        # one whole step captured once (profiling off), replayed in the timed pass
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
-    def timed_steps(only=None, profile=True):
+    def timed_steps(only=None, profile=True, replay=False):
         """K steps, each bracketed by events on the launching stream, L2
         flushed between steps outside the events; the library also records
         CUDA events around its kernel launches (all of them, or only kernel
@@ -391,7 +411,10 @@ def main():
         for i in range(args.steps):
             flush.zero_()
             evs[i][0].record(stream)
-            step()
+            if replay:
+                graph.replay()
+            else:
+                step()
             evs[i][1].record(stream)
         torch.cuda.synchronize()
         if world > 1:
@@ -411,12 +434,20 @@ def main():
     # every kernel (per-kernel table; event records between launches
     # serialise them, and under sustained tensor load the power limit lowers
     # the clock after some 50 ms, so pass 2 runs slower).
+    # With --cuda-graph the headline pass replays the captured step (no
+    # library events inside it) and the dominant kernel is timed in an extra
+    # eager pass right after.
     dom = warm_dominant
     if sampler:
         sampler.window(True)
-    step_ms, dom_prof = timed_steps(only=dom)
+    if graph is not None:
+        step_ms, _ = timed_steps(profile=False, replay=True)
+    else:
+        step_ms, dom_prof = timed_steps(only=dom)
     if sampler:
         sampler.window(False)
+    if graph is not None:
+        _, dom_prof = timed_steps(only=dom)
     total_ms = sum(step_ms)
     prof_step_ms, prof = timed_steps()
 

@@ -289,6 +289,7 @@ def workload_config(wl, args):
             "router_linear": bool(getattr(args, "router_linear", False)),
             "gather_fused": bool(getattr(args, "gather_fused", False)),
             "cuda_graph": bool(getattr(args, "cuda_graph", False)),
+            "dw_dtype": "f32" if getattr(args, "dw_f32", False) else "bf16",
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -305,6 +306,8 @@ def main():
                     help="capture one whole step in a CUDA graph after warm-up and time its replays")
     ap.add_argument("--gather-fused", action="store_true",
                     help="GEMMs read X / dY rows by token (no Xp / dYp copies) instead of the permuted copies")
+    ap.add_argument("--dw-f32", action="store_true",
+                    help="weight gradients written as fp32 (the wgrad accumulators unrounded) instead of bf16")
     ap.add_argument("--router-linear", action="store_true",
                     help="include the router Linear (logits = X W_r^T and its backward) in the step")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -348,7 +351,8 @@ def main():
     if rl and wl.zipf_s:
         ap.error("--router-linear: the stress workloads' logit bias has no router-weight form")
     gf = args.gather_fused
-    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl, gather=gf)
+    bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl, gather=gf,
+                          dw_f32=args.dw_f32)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

@@ -202,6 +202,29 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_layer_bwd with fp32 weight gradients: dW_gu [E,2I,H] and dW_d [E,H,I]
+ * are fp32, the wgrad GEMMs' fp32 accumulators stored without rounding
+ * (moe_layer_bwd rounds the same accumulators to bf16, so rounding this
+ * output to bf16 gives moe_layer_bwd's dW bit for bit).
+ * accumulate != 0: dW_gu += gradient and dW_d += gradient (one fp32 add per
+ * element, each element written by one thread; experts with no rows leave
+ * their dW unchanged) -- a gradient summed over micro-batches in fp32.
+ * accumulate == 0: dW = gradient, zeros for experts with no rows.
+ * dW_gu / dW_d 16-byte aligned, contiguous. Every other argument, the
+ * workspace (moe_layer_bwd_workspace_bytes) and the error codes are those
+ * of moe_layer_bwd.
+ * Source: "Optimizing Mixture of Experts Models" (axolotl issue #3155),
+ * expert weights [num_experts, 2*intermediate_dim, hidden_dim] and
+ * [num_experts, hidden_dim, intermediate_dim]; the pages train in bf16 and
+ * leave the gradient's precision open.
+ */
+int moe_layer_bwd_dw_f32(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                         const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                         const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                         const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, float* dW_gu, float* dW_d,
+                         int accumulate, float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Gather-fused variants -- the same results as moe_experts_fwd and
  * moe_layer_bwd, reading the activations in token order: the GEMMs load the
  * rows of X [T,H] (and of dY [T,H]) by token index t = sorted_pair[r] / k
@@ -226,6 +249,14 @@ int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_sa
                     const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
                     const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
                     float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_layer_bwd_dw_f32 with X [T,H] in token order in place of Xp;
+ * ws >= moe_layer_bwd_x_workspace_bytes(...). */
+int moe_layer_bwd_x_dw_f32(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
+                           const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                           const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                           const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, float* dW_gu, float* dW_d,
+                           int accumulate, float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Router Linear -- logits = X W_r^T and its backward, on the tensor cores.

@@ -39,6 +39,10 @@ _SIGNATURES = {
     "moe_layer_bwd": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
     "moe_layer_bwd_x_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "moe_layer_bwd_x": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
+    "moe_layer_bwd_dw_f32": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 5 + [_c_int, _c_void, _c_void,
+                                                                                     _c_size, _c_void]),
+    "moe_layer_bwd_x_dw_f32": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 5 + [_c_int, _c_void, _c_void,
+                                                                                       _c_size, _c_void]),
     "moe_router_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_router_fwd": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void,
                                 _c_void, _c_void, _c_size, _c_void]),
@@ -182,25 +186,40 @@ def moe_combine(O, pair_pos, T, k, Y=None, stream=None):
 
 
 def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
-                  W_gu, W_d, out=None, ws=None, stream=None, gather=False):
-    """gather=True: `Xp` is X [T, H] in token order (moe_layer_bwd_x)."""
+                  W_gu, W_d, out=None, ws=None, stream=None, gather=False, dw_dtype=torch.bfloat16,
+                  accumulate=False):
+    """gather=True: `Xp` is X [T, H] in token order (moe_layer_bwd_x).
+    dw_dtype=torch.float32: fp32 weight gradients (moe_layer_bwd_dw_f32);
+    accumulate=True then adds them to out["dW_gu"] / out["dW_d"]."""
     H = W_gu.shape[2]
     I = W_d.shape[2]
     dev = dY.device
+    f32 = dw_dtype == torch.float32
+    if not f32 and dw_dtype != torch.bfloat16:
+        raise ValueError(f"dw_dtype must be bfloat16 or float32, not {dw_dtype}")
+    if accumulate and not (f32 and out and "dW_gu" in out and "dW_d" in out):
+        raise ValueError("accumulate needs float32 dW_gu and dW_d given in `out`")
     o = dict(out or {})
     o.setdefault("dX", torch.empty(T, H, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dW_d", torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=dw_dtype, device=dev))
+    o.setdefault("dW_d", torch.empty(E, H, I, dtype=dw_dtype, device=dev))
     o.setdefault("dlogits", torch.empty(T, E, dtype=torch.float32, device=dev))
+    _need(o["dW_gu"], dw_dtype, (E, 2 * I, H), "dW_gu")
+    _need(o["dW_d"], dw_dtype, (E, H, I), "dW_d")
     query = lib().moe_layer_bwd_x_workspace_bytes if gather else lib().moe_layer_bwd_workspace_bytes
     need = query(T, E, k, H, I, 1 if gu_save is None else 0)
     if ws is None:
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     name = "moe_layer_bwd_x" if gather else "moe_layer_bwd"
-    _check(name, getattr(lib(), name)(
-        _ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
-        _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]),
-        _ptr(o["dW_gu"]), _ptr(o["dW_d"]), _ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream)))
+    head = (_ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
+            _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]),
+            _ptr(o["dW_gu"]), _ptr(o["dW_d"]))
+    tail = (_ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream))
+    if f32:
+        name += "_dw_f32"
+        _check(name, getattr(lib(), name)(*head, 1 if accumulate else 0, *tail))
+    else:
+        _check(name, getattr(lib(), name)(*head, *tail))
     return o
 
 

@@ -144,6 +144,8 @@ struct GemmParams {
   int gather_cols;
   int tails;                  // row-grouped kinds: segment tails of 1..128 rows go to the one-CTA instance
   int wait_at_end;            // pair instance launched after a one-CTA instance: wait for it at the end
+  float* out_f32;             // wgrad: fp32 output in place of `out` (NULL: bf16 to `out`), same strides
+  int accumulate;             // wgrad with out_f32: out_f32 += acc (fp32 add) instead of out_f32 = acc
 };
 
 template <int CG>
@@ -265,6 +267,41 @@ __device__ __forceinline__ void emit_chunk(uint8_t* stg, const float (&v)[32], u
     if (r < wrows && col < ncols) store16(base + (row0 + r) * ld + col, read_piece(stg, r, tr_q));
   }
   __syncwarp();
+}
+
+// fp32 variant of emit_chunk: the chunk's 32 columns go through the staging
+// buffer as two halves of 16 fp32 (64 bytes per row, the bf16 chunk's
+// footprint and swizzle); in the transposed domain lane l then owns rows
+// 8*i + l/4 and columns 4*(l%4)..+3 of the half. accumulate: base += v.
+__device__ __forceinline__ void emit_chunk_f32(uint8_t* stg, const uint32_t (&a)[32], float* base, int64_t row0,
+                                               int64_t ld, int col0, int ncols, int wrows, int tr_row, int tr_q,
+                                               int lane, bool accumulate) {
+  uint8_t* rp = stg + lane * kStageStrideBytes;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      *reinterpret_cast<uint4*>(rp + 16 * (m ^ sw)) =
+          make_uint4(a[16 * half + 4 * m], a[16 * half + 4 * m + 1], a[16 * half + 4 * m + 2], a[16 * half + 4 * m + 3]);
+    __syncwarp();
+    const int col = col0 + 16 * half + 4 * tr_q;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + tr_row;
+      if (r < wrows && col < ncols) {
+        float4* dst = reinterpret_cast<float4*>(base + (row0 + r) * ld + col);
+        const uint4 u = read_piece(stg, r, tr_q);
+        float4 v = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+        if (accumulate) {
+          const float4 o = *dst;
+          v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+        }
+        *dst = v;
+      }
+    }
+    __syncwarp();
+  }
 }
 
 // dgrad-down epilogue operands in the transposed domain: for rows 8*i + tr_row
@@ -709,17 +746,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       // first output row of this warp: permuted row (row-grouped) or dW row (wgrad)
       const int64_t wrow0 = kWgrad ? static_cast<int64_t>(ti.m_blk) * kBM + cta_row0
                                    : static_cast<int64_t>(ti.row0) + cta_row0;
-      uint16_t* out_base = kWgrad ? p.out + ti.e * p.out_expert_stride : p.out;
+      uint16_t* out_base = kWgrad ? (p.out_f32 != nullptr ? nullptr : p.out + ti.e * p.out_expert_stride) : p.out;
+      float* out_f32 = kWgrad && p.out_f32 != nullptr ? p.out_f32 + ti.e * p.out_expert_stride : nullptr;
       const int ch0 = half * kChunks;  // first 32-column chunk of this warp
       if constexpr (kWgrad) {
-        if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero
+        if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero (unchanged if accumulating)
+          if (out_f32 != nullptr && p.accumulate) continue;
           for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
             const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = i * 8 + tr_row;
-              if (r < wrows && col < p.N)
-                *reinterpret_cast<uint4*>(out_base + (wrow0 + r) * p.out_ld + col) = make_uint4(0, 0, 0, 0);
+              if (r < wrows && col < p.N) {
+                if (out_f32 != nullptr) {
+                  float4* dst = reinterpret_cast<float4*>(out_f32 + (wrow0 + r) * p.out_ld + col);
+                  dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                  *reinterpret_cast<uint4*>(out_base + (wrow0 + r) * p.out_ld + col) = make_uint4(0, 0, 0, 0);
+                }
+              }
             }
           }
           continue;
@@ -847,6 +893,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, a1);
           tmem_ld_wait();
           const int col0 = ti.n_blk * kBN + ch * 32;
+          if (kWgrad && out_f32 != nullptr) {  // fp32 weight gradient: the accumulator unrounded
+            const bool accum = p.accumulate != 0;
+            if (col0 < p.N)
+              emit_chunk_f32(stg, a0, out_f32, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane, accum);
+            if (col0 + 32 < p.N)
+              emit_chunk_f32(stg, a1, out_f32, wrow0, p.out_ld, col0 + 32, p.N, wrows, tr_row, tr_q, lane, accum);
+            continue;
+          }
           float v[32];
           if (col0 < p.N) {  // warp-uniform
 #pragma unroll

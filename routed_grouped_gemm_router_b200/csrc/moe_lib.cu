@@ -655,14 +655,22 @@ size_t moe_layer_bwd_x_workspace_bytes(int T, int E, int k, int H, int I, int re
 
 namespace moe {
 namespace {
+void set_dw_out(GemmParams& p, void* dW, bool dw_f32, bool accumulate) {
+  p.out = dw_f32 ? nullptr : static_cast<uint16_t*>(dW);
+  p.out_f32 = dw_f32 ? static_cast<float*>(dW) : nullptr;
+  p.accumulate = dw_f32 && accumulate ? 1 : 0;
+}
+
 // The layer's backward. gather: `src` is X [T, H] in token order and the
 // GEMMs that read X or dY rows gather them (no dYp copy, no gather kernel);
 // otherwise `src` is Xp [P, H] and dY is first gathered into dYp.
+// dw_f32: dW_gu / dW_d are fp32 (the wgrad accumulators unrounded), else
+// bf16; accumulate (fp32 only): dW += the gradient instead of dW = it.
 int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const moe_bf16* gu_save,
                    const moe_bf16* h, const float* probs, const int32_t* topk_idx, const float* topk_w,
                    const int32_t* offsets, const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k,
-                   int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu,
-                   moe_bf16* dW_d, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                   int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, void* dW_gu, void* dW_d,
+                   bool dw_f32, bool accumulate, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
@@ -677,9 +685,11 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
-  const size_t dw_gu_bytes = static_cast<size_t>(E) * 2 * I * H * 2;
-  const size_t dw_d_bytes = static_cast<size_t>(E) * H * I * 2;
+  const size_t dw_elem = dw_f32 ? 4 : 2;
+  const size_t dw_gu_bytes = static_cast<size_t>(E) * 2 * I * H * dw_elem;
+  const size_t dw_d_bytes = static_cast<size_t>(E) * H * I * dw_elem;
   if (P == 0) {  // no rows: every expert is empty, all weight gradients are zero
+    if (accumulate) return MOE_OK;  // dW += 0
     if (cudaMemsetAsync(dW_gu, 0, dw_gu_bytes, stream) != cudaSuccess ||
         cudaMemsetAsync(dW_d, 0, dw_d_bytes, stream) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -799,7 +809,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wg.I = I;
     wg.m_tiles = cdiv(2 * I, kBM);
     wg.n_tiles = cdiv(H, kBN);
-    wg.out = dW_gu;
+    set_dw_out(wg, dW_gu, dw_f32, accumulate);
     wg.out_ld = H;
     wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
     const int64_t tiles = static_cast<int64_t>(E) * wg.m_tiles * wg.n_tiles;
@@ -826,7 +836,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wd.I = I;
     wd.m_tiles = cdiv(H, kBM);
     wd.n_tiles = cdiv(I, kBN);
-    wd.out = dW_d;
+    set_dw_out(wd, dW_d, dw_f32, accumulate);
     wd.out_ld = I;
     wd.out_expert_stride = static_cast<int64_t>(H) * I;
     const int64_t tiles = static_cast<int64_t>(E) * wd.m_tiles * wd.n_tiles;
@@ -858,7 +868,16 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
-                        H, I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
+                        H, I, W_gu, W_d, dX, dW_gu, dW_d, false, false, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_layer_bwd_dw_f32(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                         const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                         const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                         const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, float* dW_gu, float* dW_d,
+                         int accumulate, float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
+                        H, I, W_gu, W_d, dX, dW_gu, dW_d, true, accumulate != 0, dlogits, ws, ws_bytes, stream);
 }
 
 int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
@@ -867,7 +886,16 @@ int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_sa
                     const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d,
                     float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return layer_bwd_impl(dY, X, true, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k, H,
-                        I, W_gu, W_d, dX, dW_gu, dW_d, dlogits, ws, ws_bytes, stream);
+                        I, W_gu, W_d, dX, dW_gu, dW_d, false, false, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_layer_bwd_x_dw_f32(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,
+                           const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                           const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                           const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, float* dW_gu, float* dW_d,
+                           int accumulate, float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_bwd_impl(dY, X, true, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k, H,
+                        I, W_gu, W_d, dX, dW_gu, dW_d, true, accumulate != 0, dlogits, ws, ws_bytes, stream);
 }
 
 size_t moe_router_workspace_bytes(int T, int H, int E) {

@@ -71,22 +71,28 @@ def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, g
 
 
 def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, bufs: dict | None = None,
-             stream=None) -> dict:
-    """dX, dW_gu, dW_d, dlogits for upstream gradient dY."""
+             stream=None, accumulate: bool = False) -> dict:
+    """dX, dW_gu, dW_d, dlogits for upstream gradient dY. The weight
+    gradients are bf16, or fp32 when the buffers in bufs["grads"] are fp32
+    (``allocate(..., dw_f32=True)``); accumulate=True adds to those fp32
+    buffers instead of overwriting them."""
     b = bufs or {}
     p = st.perm
     gather = st.X is not None
+    grads = b.get("grads")
+    dw_dtype = grads["dW_gu"].dtype if grads and "dW_gu" in grads else torch.bfloat16
     return B.moe_layer_bwd(dY, st.X if gather else p["Xp"], st.gu, st.h, st.probs, st.topk_idx, st.topk_w,
                            p["offsets"], p["sorted_pair"], p["pair_pos"], st.T, st.E, st.k, W_gu, W_d,
-                           out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream, gather=gather)
+                           out=grads, ws=b.get("bwd_ws"), stream=stream, gather=gather, dw_dtype=dw_dtype,
+                           accumulate=accumulate)
 
 
 def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor,
-                  W_d: torch.Tensor, bufs: dict | None = None, stream=None) -> dict:
+                  W_d: torch.Tensor, bufs: dict | None = None, stream=None, accumulate: bool = False) -> dict:
     """``backward`` plus the router Linear's: dX gains dlogits W_r (in place)
     and the result holds dW_r = dlogits^T X."""
     b = bufs or {}
-    g = backward(st, dY, W_gu, W_d, bufs=b, stream=stream)
+    g = backward(st, dY, W_gu, W_d, bufs=b, stream=stream, accumulate=accumulate)
     dW_r, _ = B.moe_router_bwd(g["dlogits"], X, W_r, dX=g["dX"], dW_r=b.get("dW_r"), ws=b.get("router_ws"),
                                stream=stream)
     g["dW_r"] = dW_r
@@ -94,10 +100,12 @@ def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.
 
 
 def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False,
-             gather: bool = False) -> dict:
-    """Every output and workspace of one forward+backward, allocated once."""
+             gather: bool = False, dw_f32: bool = False) -> dict:
+    """Every output and workspace of one forward+backward, allocated once;
+    dw_f32: fp32 weight-gradient buffers."""
     P = T * k
     bf = torch.bfloat16
+    dwt = torch.float32 if dw_f32 else bf
     lib = B.lib()
     d = dict(
         topk_idx=torch.empty(T, k, dtype=torch.int32, device=device),
@@ -113,8 +121,8 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
         O=torch.empty(P, H, dtype=bf, device=device),
         Y=torch.empty(T, H, dtype=bf, device=device),
         grads=dict(dX=torch.empty(T, H, dtype=bf, device=device),
-                   dW_gu=torch.empty(E, 2 * I, H, dtype=bf, device=device),
-                   dW_d=torch.empty(E, H, I, dtype=bf, device=device),
+                   dW_gu=torch.empty(E, 2 * I, H, dtype=dwt, device=device),
+                   dW_d=torch.empty(E, H, I, dtype=dwt, device=device),
                    dlogits=torch.empty(T, E, dtype=torch.float32, device=device)),
         bwd_ws=torch.empty(max((lib.moe_layer_bwd_x_workspace_bytes if gather else lib.moe_layer_bwd_workspace_bytes)(
             T, E, k, H, I, 0 if save_gu else 1), 1), dtype=torch.uint8, device=device),

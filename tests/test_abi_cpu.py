@@ -58,6 +58,17 @@ def test_invalid_arguments_rejected_without_device():
     args = [p] * 10 + [4, 8, 2, 16, 16] + [p] * 6
     assert lib.moe_layer_bwd(*args, p, need - 1, NULL) == 3
     assert lib.moe_layer_bwd(*([p, p, NULL] + [p] * 7 + [4, 8, 2, 16, 16] + [p] * 6), p, need - 1, NULL) == 3
+    # fp32 weight gradients: the same checks; dW pointers must be 16-byte aligned
+    f32_args = [p] * 10 + [4, 8, 2, 16, 16] + [p] * 5
+    for name in ("moe_layer_bwd_dw_f32", "moe_layer_bwd_x_dw_f32"):
+        fn = getattr(lib, name)
+        q = (lib.moe_layer_bwd_x_workspace_bytes if "_x_" in name else lib.moe_layer_bwd_workspace_bytes)(
+            4, 8, 2, 16, 16, 0)
+        assert fn(*f32_args, 0, p, p, q - 1, NULL) == 3
+        assert fn(*f32_args, 1, p, p, q - 1, NULL) == 3
+        assert fn(*([p] * 10 + [4, 8, 2, 16, 16] + [p] * 4 + [odd]), 0, p, p, q, NULL) == 1
+        assert fn(*([p] * 10 + [4, 8, 2, 16, 16] + [p] * 3 + [NULL, p]), 1, p, p, q, NULL) == 1
+        assert fn(*([p] * 10 + [4, 8, 2, 16, 12] + [p] * 5), 0, p, p, q, NULL) == 1  # I not a multiple of 8
 
 
 def test_empty_batch_needs_no_device():

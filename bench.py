@@ -427,6 +427,11 @@ def main():
         prof = None
         if profile:
             prof = B.profile_read()
+            # effective SM clock of each GEMM, from the kernels' own cycle and
+            # nanosecond counters (NVML's clock reading does not resolve them)
+            for n in list(prof):
+                if n.startswith("gemm_"):
+                    prof[n] = prof[n] + (B.profile_read_clock(n),)
             B.profile_enable(False)
         status = B.last_device_status()
         if status != 0:
@@ -557,7 +562,8 @@ def main():
     # dominant kernel: most device time over the timed region
     kernels = {}
     launches = 0
-    for name, (ms, n) in prof.items():
+    for name, rec in prof.items():
+        ms, n = rec[0], rec[1]
         kind, work = kernel_work(name, wl)
         avg_ms = ms / n
         launches += n
@@ -566,6 +572,8 @@ def main():
                          "bound": kind,
                          "achieved": rate / 1e12 if kind == "tensor" else rate / 1e9,
                          "unit": "TFLOP/s" if kind == "tensor" else "GB/s"}
+        if len(rec) > 2:
+            kernels[name]["sm_mhz_in_kernel"] = round(rec[2])
     kind, work = kernel_work(dom, wl)
     avg_s = dom_prof[dom][0] / dom_prof[dom][1] * 1e-3
     if kind == "tensor":
@@ -578,6 +586,12 @@ def main():
         achieved = work / avg_s / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    if len(dom_prof[dom]) > 2:
+        roof["sm_mhz_in_kernel"] = round(dom_prof[dom][2])
+        if clocks is not None:
+            # NVML's reading is a coarse average: the kernel's own counters
+            # give the clock it really ran at in the headline pass
+            clocks["dominant_gemm_sm_mhz_in_kernel"] = round(dom_prof[dom][2])
     roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name), "algorithmic_per_launch": work,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 

@@ -325,6 +325,13 @@ int moe_profile_enable(int on);
  * disturbance of the launch stream. MOE_ERR_INVALID_ARG for an unknown name. */
 int moe_profile_only(const char* name);
 int moe_profile_read(const char* name, double* total_ms, int* launches);
+/* Effective SM clock (MHz) of grouped-GEMM kernel `name` over the launches
+ * recorded since moe_profile_enable(1): SM cycles counted by each CTA's MMA
+ * issuer over its main loop, divided by the global nanoseconds of the same
+ * interval. It shows the clock the kernel really ran at (the power limit
+ * lowers it). 0 when nothing was recorded or `name` is not a GEMM.
+ * Synchronises the device. MOE_ERR_INVALID_ARG for an unknown name. */
+int moe_profile_read_clock(const char* name, double* sm_mhz);
 /* Name of kernel slot i (0-based), NULL past the last one. */
 const char* moe_profile_kernel_name(int i);
 

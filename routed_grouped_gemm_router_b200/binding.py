@@ -53,6 +53,7 @@ _SIGNATURES = {
     "moe_profile_only": (_c_int, [ctypes.c_char_p]),
     "moe_profile_read": (_c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_int)]),
     "moe_profile_kernel_name": (ctypes.c_char_p, [_c_int]),
+    "moe_profile_read_clock": (_c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)]),
 }
 
 
@@ -302,3 +303,11 @@ def profile_read() -> dict:
         if cnt.value:
             out[n] = (ms.value, cnt.value)
     return out
+
+
+def profile_read_clock(name: str) -> float:
+    """Effective SM clock (MHz) of GEMM kernel `name` over its recorded
+    launches, from the kernel's own cycle and nanosecond counters (0: none)."""
+    mhz = ctypes.c_double()
+    _check("moe_profile_read_clock", lib().moe_profile_read_clock(name.encode(), ctypes.byref(mhz)))
+    return mhz.value

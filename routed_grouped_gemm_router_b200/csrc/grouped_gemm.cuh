@@ -146,6 +146,7 @@ struct GemmParams {
   int wait_at_end;            // pair instance launched after a one-CTA instance: wait for it at the end
   float* out_f32;             // wgrad: fp32 output in place of `out` (NULL: bf16 to `out`), same strides
   int accumulate;             // wgrad with out_f32: out_f32 += acc (fp32 add) instead of out_f32 = acc
+  unsigned long long* clock_acc;  // profiling (NULL: off): [0] += SM cycles, [1] += ns of each MMA issuer's loop
 };
 
 template <int CG>
@@ -655,6 +656,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       int stage = 0;
       uint32_t phase = 0;
       int tcount = 0;
+      // effective SM clock over the main loop (profiling only): SM cycles
+      // against global nanoseconds; the power limit lowers the first
+      const long long clk0 = clock64();
+      const unsigned long long ns0 = globaltimer_ns();
       for (int t = pair; t < total_tiles && !*s_abort; t += num_pairs) {
         const TileInfo ti = decode_tile<KIND, CG>(t, p, s_off, s_tstart);
         if (ti.num_kb == 0) continue;  // empty expert (wgrad): the epilogues write zeros
@@ -711,6 +716,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         }
         __syncwarp();
         ++tcount;
+      }
+      if (p.clock_acc != nullptr && lane == 0) {
+        atomicAdd(p.clock_acc, static_cast<unsigned long long>(clock64() - clk0));
+        atomicAdd(p.clock_acc + 1, globaltimer_ns() - ns0);
       }
       // all MMAs of the pair must finish before TMEM is released
       if (lane == 0) {

@@ -177,6 +177,21 @@ struct Profiler {
 };
 Profiler g_prof;
 
+// Per-slot effective SM clock of the GEMMs while profiling: [slot][0] SM
+// cycles, [slot][1] nanoseconds, summed over the MMA issuers' main loops.
+// A static device array: profiling allocates no device memory.
+__device__ unsigned long long g_gemm_clock[kProfSlots][2];
+
+// Device address of the slot's clock counters when that slot is being
+// profiled, else NULL (the kernels then skip the accounting).
+unsigned long long* gemm_clock_slot(int slot) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.on || (g_prof.only >= 0 && g_prof.only != slot)) return nullptr;
+  void* base = nullptr;
+  if (cudaGetSymbolAddress(&base, g_gemm_clock) != cudaSuccess) return nullptr;
+  return static_cast<unsigned long long*>(base) + 2 * slot;
+}
+
 // Brackets one kernel launch with events on its stream when profiling is on.
 struct ProfScope {
   int slot;
@@ -218,6 +233,7 @@ int launch_gemm_instance(const GemmParams& p, int grid, cudaStream_t s) {
 template <int KIND, int GATHER = kNoGather>
 int launch_gemm(GemmParams p, int grid, cudaStream_t s, int slot, int tail_ctas = 0, int num_sms = 0) {
   ProfScope ps(slot, s);
+  p.clock_acc = gemm_clock_slot(slot);
   if constexpr (KIND != kBwdWgrad && GATHER == kNoGather) {
     if (kTailTiles && tail_ctas > 0) {
       p.tails = 1;
@@ -1050,7 +1066,27 @@ int moe_profile_enable(int on) {
   g_prof.clear();
   g_prof.on = (on != 0);
   g_prof.only = -1;
+  if (on) {
+    void* base = nullptr;
+    if (cudaGetSymbolAddress(&base, g_gemm_clock) != cudaSuccess ||
+        cudaMemset(base, 0, sizeof(unsigned long long) * 2 * kProfSlots) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   return MOE_OK;
+}
+
+int moe_profile_read_clock(const char* name, double* sm_mhz) {
+  if (name == nullptr || sm_mhz == nullptr) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < kProfSlots; ++i) {
+    if (std::strcmp(name, kProfNames[i]) != 0) continue;
+    unsigned long long c[kProfSlots][2];
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(c, g_gemm_clock, sizeof(c)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    *sm_mhz = c[i][1] > 0 ? 1e3 * static_cast<double>(c[i][0]) / static_cast<double>(c[i][1]) : 0.0;
+    return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
 }
 
 int moe_profile_only(const char* name) {

@@ -83,6 +83,9 @@ def test_profile_names():
     names = B.profile_kernel_names()
     assert "gemm_fwd_gate_up" in names and "router_bwd" in names
     assert len(names) == len(set(names))
+    d = ctypes.c_double()
+    assert B.lib().moe_profile_read_clock(b"no_such_kernel", ctypes.byref(d)) == 1
+    assert B.lib().moe_profile_read_clock(None, ctypes.byref(d)) == 1
 
 
 def test_router_linear_arguments_rejected_without_device():

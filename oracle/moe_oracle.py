@@ -26,6 +26,9 @@ Sources (page title, then the part of the page):
   * modelopt ``moe`` helpers, ``a2a_moe`` *Flow*: expand (token, expert) pairs,
     run the experts, then weight each result by its routing weight and sum each
     token's top-k results.
+  * fused-MoE Triton project summary (sourcepulse), *Highlighted Details*:
+    LoRA on the fused expert weights (``lora_*`` functions; the update itself
+    is the published LoRA form W + scale B A).
 
 Readings where the pages are silent (each is also listed in the design notes):
   1. top-k is taken on the fp32 logits (softmax is strictly increasing, so the
@@ -36,6 +39,8 @@ Readings where the pages are silent (each is also listed in the design notes):
   4. the routing weight multiplies the expert output before the per-token sum.
   5. backward: the top-k selection is a constant; gradients flow through
      softmax -> gather -> renormalisation (what autograd of that chain gives).
+  6. LoRA: one adapter per expert on each stacked weight (gate|up fused), one
+     scale; the base weights are frozen (their gradient is still returned).
 
 Notation: T tokens, H hidden, E experts, k top-k, I expert intermediate size,
 P = T*k pairs, pair id q = t*k + j (j = rank of the expert in token t's top-k).
@@ -240,6 +245,48 @@ def router_logits_backward(dlogits, X, W_r):
     (the layer's dX is the experts' dX plus this)."""
     dl = _f64(dlogits)
     return dl.T @ _f64(X), dl @ _f64(W_r)
+
+
+# ------------------------------------------------------------------ LoRA adapters
+# Source: fused-MoE Triton project summary (sourcepulse), *Highlighted
+# Details*: LoRA (and QLoRA) on the fused expert weights, with conversion
+# between the fused and the unfused adapter formats. The pages give no
+# formulas; the adapter is the published LoRA update (Hu et al., "LoRA:
+# Low-Rank Adaptation of Large Language Models", 2021): a frozen weight W
+# [out, in] is used as W + scale * B A with A [r, in], B [out, r] trainable.
+# Reading: one adapter per expert on each stacked weight -- A_gu [E, r, H] and
+# B_gu [E, 2I, r] on W_gu (the fused gate|up format), A_d [E, r, I] and B_d
+# [E, H, r] on W_d -- and one scale for all of them.
+def lora_effective_weights(W_gu, W_d, A_gu, B_gu, A_d, B_d, scale: float):
+    """The weights the layer uses: W_gu[e] + scale B_gu[e] A_gu[e] and
+    W_d[e] + scale B_d[e] A_d[e], in float64."""
+    W_gu_eff = _f64(W_gu) + scale * np.einsum("eor,eri->eoi", _f64(B_gu), _f64(A_gu))
+    W_d_eff = _f64(W_d) + scale * np.einsum("eor,eri->eoi", _f64(B_d), _f64(A_d))
+    return W_gu_eff, W_d_eff
+
+
+def lora_layer_forward(logits, X, W_gu, W_d, k: int, A_gu, B_gu, A_d, B_d, scale: float) -> dict:
+    """``layer_forward`` with the adapted weights (route, permute, SwiGLU
+    experts, weighted combine are unchanged)."""
+    W_gu_eff, W_d_eff = lora_effective_weights(W_gu, W_d, A_gu, B_gu, A_d, B_d, scale)
+    fwd = layer_forward(logits, X, W_gu_eff, W_d_eff, k)
+    fwd["W_gu_eff"], fwd["W_d_eff"] = W_gu_eff, W_d_eff
+    return fwd
+
+
+def lora_layer_backward(fwd: dict, dY, X, k: int, A_gu, B_gu, A_d, B_d, scale: float) -> dict:
+    """Backward of ``lora_layer_forward``. dX and dlogits are those of the
+    layer with the adapted weights; the gradient reaching a weight, G = dL/dW
+    (the same for the frozen W and for W + scale B A), gives by the chain rule
+    of W + scale B A: dA = scale B^T G and dB = scale G A^T, per expert."""
+    g = layer_backward(fwd, dY, X, fwd["W_gu_eff"], fwd["W_d_eff"], k)
+    sc = float(scale)
+    G_gu, G_d = g["dW_gu"], g["dW_d"]
+    g["dA_gu"] = sc * np.einsum("eor,eoi->eri", _f64(B_gu), G_gu)
+    g["dB_gu"] = sc * np.einsum("eoi,eri->eor", G_gu, _f64(A_gu))
+    g["dA_d"] = sc * np.einsum("eor,eoi->eri", _f64(B_d), G_d)
+    g["dB_d"] = sc * np.einsum("eoi,eri->eor", G_d, _f64(A_d))
+    return g
 
 
 # ----------------------------------------------------------- sampled (large sizes)

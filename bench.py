@@ -42,13 +42,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # Algorithmic work per launch of each kernel, as a function of the workload:
 # GEMMs in flops (bf16 tensor cores), memory kernels in bytes (HBM).
-def kernel_work(name, wl):
+def kernel_work(name, wl, lora_r=0):
     T, H, E, k, I, P = wl.T, wl.H, wl.E, wl.k, wl.I, wl.P
+    r = lora_r
     flops = {
-        "gemm_fwd_gate_up": 4.0 * H * I * P, "gemm_fwd_down": 2.0 * H * I * P,
-        "gemm_recompute_gate_up": 4.0 * H * I * P,
-        "gemm_bwd_dgrad_down": 2.0 * H * I * P, "gemm_bwd_dgrad_gate_up": 4.0 * H * I * P,
+        # with adapters of rank r the row-grouped GEMMs also run the adapter
+        # term as r more K columns ([act | Z] [W | B])
+        "gemm_fwd_gate_up": 4.0 * H * I * P + 4.0 * I * r * P, "gemm_fwd_down": 2.0 * H * I * P + 2.0 * H * r * P,
+        "gemm_recompute_gate_up": 4.0 * H * I * P + 4.0 * I * r * P,
+        "gemm_bwd_dgrad_down": 2.0 * H * I * P + 2.0 * I * r * P,
+        "gemm_bwd_dgrad_gate_up": 4.0 * H * I * P + 2.0 * H * r * P,
         "gemm_bwd_wgrad_gate_up": 4.0 * H * I * P, "gemm_bwd_wgrad_down": 2.0 * H * I * P,
+        # adapter products (useful flops; their tiles are 256 wide in r)
+        "gemm_lora_z_gate_up": 2.0 * H * r * P, "gemm_lora_z_down": 2.0 * I * r * P,
+        "gemm_lora_v_down": 2.0 * H * r * P, "gemm_lora_v_gate_up": 4.0 * I * r * P,
+        "gemm_lora_da_gate_up": 2.0 * H * r * P, "gemm_lora_db_gate_up": 4.0 * I * r * P,
+        "gemm_lora_da_down": 2.0 * I * r * P, "gemm_lora_db_down": 2.0 * H * r * P,
     }
     if name in flops:
         return "tensor", flops[name]
@@ -64,6 +73,7 @@ def kernel_work(name, wl):
         "gemm_router_logits": T * H * 2 + E * H * 4 + T * E * 4,
         "gemm_router_wgrad": T * H * 2 + T * E * 4 + E * H * 4, "router_sum_splits": 2 * E * H * 4,
         "gemm_router_dgrad": T * E * 4 + E * H * 4 + 2 * T * H * 2,
+        "lora_weight_rows": 2 * P * r * 2 + P * 8,
     }
     return "hbm", float(nbytes.get(name, 0))
 
@@ -199,9 +209,15 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_step(inp_sub, k, backward, router=False):
+def oracle_step(inp_sub, k, backward, router=False, lora=None):
     from oracle import moe_oracle as orc
     logits = orc.router_logits(inp_sub.X, inp_sub.W_r) if router else inp_sub.logits
+    if lora is not None:
+        a = [lora[n] for n in ("A_gu", "B_gu", "A_d", "B_d")] + [lora["scale"]]
+        fwd = orc.lora_layer_forward(logits, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k, *a)
+        if backward:
+            orc.lora_layer_backward(fwd, inp_sub.dY, inp_sub.X, k, *a)
+        return
     fwd = orc.layer_forward(logits, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
     if backward:
         bwd = orc.layer_backward(fwd, inp_sub.dY, inp_sub.X, inp_sub.W_gu, inp_sub.W_d, k)
@@ -209,7 +225,7 @@ def oracle_step(inp_sub, k, backward, router=False):
             orc.router_logits_backward(bwd["dlogits"], inp_sub.X, inp_sub.W_r)
 
 
-def cpu_sample(inp, wl, target_s, router=False):
+def cpu_sample(inp, wl, target_s, router=False, lora=None):
     """The first T_s tokens of the batch (all E experts), T_s sized so one
     oracle fwd+bwd takes about target_s seconds on the host cores."""
     import copy
@@ -222,18 +238,42 @@ def cpu_sample(inp, wl, target_s, router=False):
 
     ts = min(wl.T, 64)
     t0 = time.perf_counter()
-    oracle_step(sub(ts), wl.k, wl.backward, router)
+    oracle_step(sub(ts), wl.k, wl.backward, router, lora)
     dt = time.perf_counter() - t0
     while ts < wl.T and dt < target_s / 4:
         ts = min(wl.T, ts * 4)
         t0 = time.perf_counter()
-        oracle_step(sub(ts), wl.k, wl.backward, router)
+        oracle_step(sub(ts), wl.k, wl.backward, router, lora)
         dt = time.perf_counter() - t0
     return sub(ts), ts
 
 
-def step_flops(wl):
+def step_flops(wl, lora_r=0):
+    """Useful flops of one step. With adapters of rank r the base weights
+    are frozen: the backward has the dgrad GEMMs (6 H I per pair) but no base
+    weight gradients, and every adapter product counts (2 r (6H + 9I) per
+    pair over the forward and backward)."""
+    if lora_r:
+        P, H, I = wl.P, wl.H, wl.I
+        base = 6.0 * H * I * P * (2 if wl.backward else 1)
+        return base + 2.0 * P * lora_r * ((6 * H + 9 * I) if wl.backward else (2 * H + 3 * I))
     return wl.flops_fwd() + (wl.flops_bwd() if wl.backward else 0.0)
+
+
+def lora_np(wl, args):
+    """The bench's adapters as float64 arrays for the oracle."""
+    d = lora_inputs(wl, args.lora, args.seed)
+    out = {n: d[n].double().numpy() for n in ("A_gu", "B_gu", "A_d", "B_d")}
+    out["scale"] = d["scale"]
+    return out
+
+
+def lora_inputs(wl, r, seed, scale=2.0):
+    """Seeded rank-r adapters for the workload (bf16; scale = alpha / r)."""
+    from routed_grouped_gemm_router_b200.inputs import make_lora
+    d = make_lora(wl.E, wl.H, wl.I, r, seed=seed + 1000)
+    d["scale"] = scale
+    return d
 
 
 def world_info():
@@ -260,15 +300,16 @@ def run_reference(args, wl, rank):
     if rank != 0:
         return
     inp = make_inputs(wl, seed=args.seed)
-    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s, router=args.router_linear)
+    lo = lora_np(wl, args) if args.lora else None
+    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s, router=args.router_linear, lora=lo)
     sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
     for _ in range(args.warmup):
-        oracle_step(sample, wl.k, wl.backward, args.router_linear)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(sample, wl.k, wl.backward, args.router_linear)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
     dt = (time.perf_counter() - t0) / args.steps
-    value = step_flops(sub_wl) / dt / 1e12
+    value = step_flops(sub_wl, args.lora) / dt / 1e12
     desc = f"first {ts} of {wl.T} tokens, all {wl.E} experts, {'fwd+bwd' if wl.backward else 'fwd'} in float64"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -285,11 +326,14 @@ def run_reference(args, wl, rank):
 def workload_config(wl, args):
     return {"workload": f"{wl.name} MoE layer {'fwd+bwd' if wl.backward else 'fwd'}: T={wl.T} H={wl.H} "
                         f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else "")
-                        + (" + router Linear (fp32, on the GPU)" if getattr(args, "router_linear", False) else ""),
+                        + (" + router Linear (fp32, on the GPU)" if getattr(args, "router_linear", False) else "")
+                        + (f" + LoRA rank {args.lora} on the expert weights (base frozen)"
+                           if getattr(args, "lora", 0) else ""),
             "router_linear": bool(getattr(args, "router_linear", False)),
             "gather_fused": bool(getattr(args, "gather_fused", False)),
             "cuda_graph": bool(getattr(args, "cuda_graph", False)),
             "dw_dtype": "f32" if getattr(args, "dw_f32", False) else "bf16",
+            "lora_rank": int(getattr(args, "lora", 0)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -306,6 +350,8 @@ def main():
                     help="capture one whole step in a CUDA graph after warm-up and time its replays")
     ap.add_argument("--gather-fused", action="store_true",
                     help="GEMMs read X / dY rows by token (no Xp / dYp copies) instead of the permuted copies")
+    ap.add_argument("--lora", type=int, default=0, metavar="R",
+                    help="LoRA adapters of rank R on the expert weights; base weights frozen (no dW GEMMs)")
     ap.add_argument("--dw-f32", action="store_true",
                     help="weight gradients written as fp32 (the wgrad accumulators unrounded) instead of bf16")
     ap.add_argument("--router-linear", action="store_true",
@@ -351,20 +397,36 @@ def main():
     if rl and wl.zipf_s:
         ap.error("--router-linear: the stress workloads' logit bias has no router-weight form")
     gf = args.gather_fused
+    lr = args.lora
+    if lr and (rl or gf or args.dw_f32):
+        ap.error("--lora runs the permuted-operand layer on the caller's logits with frozen base weights")
+    lora = None
+    if lr:
+        lora = {n: (t.to(dev) if torch.is_tensor(t) else t) for n, t in lora_inputs(wl, lr, args.seed).items()}
     bufs = layer.allocate(wl.T, wl.E, wl.k, wl.H, wl.I, dev, save_gu=True, router=rl, gather=gf,
-                          dw_f32=args.dw_f32)
+                          dw_f32=args.dw_f32, lora_r=lr)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def run_step(X_, logits_, dY_, b):
+        """One forward (+ backward) through the public API; (state, grads)."""
+        g = None
         if rl:
-            st = layer.forward_from_x(X, W_r, W_gu, W_d, wl.k, bufs=bufs, gather=gf)
+            st = layer.forward_from_x(X_, W_r, W_gu, W_d, wl.k, bufs=b, gather=gf)
             if wl.backward:
-                layer.backward_to_x(st, dY, X, W_r, W_gu, W_d, bufs=bufs)
-            return
-        st = layer.forward(logits, X, W_gu, W_d, wl.k, bufs=bufs, gather=gf)
-        if wl.backward:
-            layer.backward(st, dY, W_gu, W_d, bufs=bufs)
+                g = layer.backward_to_x(st, dY_, X_, W_r, W_gu, W_d, bufs=b)
+        elif lr:
+            st = layer.forward_lora(logits_, X_, W_gu, W_d, wl.k, lora, bufs=b)
+            if wl.backward:
+                g = layer.backward_lora(st, dY_, W_gu, W_d, bufs=b)
+        else:
+            st = layer.forward(logits_, X_, W_gu, W_d, wl.k, bufs=b, gather=gf)
+            if wl.backward:
+                g = layer.backward(st, dY_, W_gu, W_d, bufs=b)
+        return st, g
+
+    def step():
+        run_step(X, logits, dY, bufs)
 
     for i in range(args.warmup):
         if i == args.warmup - 1:
@@ -511,14 +573,7 @@ def main():
                     upload((i + 1) % 2)
                 stream.wait_event(ev_in[b])
                 stream.wait_event(ev_copied[b])
-                if rl:
-                    st = layer.forward_from_x(din[b]["X"], W_r, W_gu, W_d, wl.k, bufs=obufs[b], gather=gf)
-                    if wl.backward:
-                        g = layer.backward_to_x(st, din[b]["dY"], din[b]["X"], W_r, W_gu, W_d, bufs=obufs[b])
-                else:
-                    st = layer.forward(din[b]["logits"], din[b]["X"], W_gu, W_d, wl.k, bufs=obufs[b], gather=gf)
-                    if wl.backward:
-                        g = layer.backward(st, din[b]["dY"], W_gu, W_d, bufs=obufs[b])
+                st, g = run_step(din[b]["X"], din[b]["logits"], din[b]["dY"], obufs[b])
                 ev_used[b].record(stream)
                 ev_out[b].record(stream)
                 with torch.cuda.stream(down):
@@ -553,7 +608,7 @@ def main():
             dist.destroy_process_group()
         return
 
-    flops = step_flops(wl)
+    flops = step_flops(wl, lr)
     ms_per_step = total_ms / args.steps
     value = aggregate_tflops(world, flops, args.steps, total_ms)
     e2e_value = aggregate_tflops(world, flops, args.steps, e2e_ms) if e2e_ms else None
@@ -564,7 +619,7 @@ def main():
     launches = 0
     for name, rec in prof.items():
         ms, n = rec[0], rec[1]
-        kind, work = kernel_work(name, wl)
+        kind, work = kernel_work(name, wl, lr)
         avg_ms = ms / n
         launches += n
         rate = work / (avg_ms * 1e-3)
@@ -574,7 +629,7 @@ def main():
                          "unit": "TFLOP/s" if kind == "tensor" else "GB/s"}
         if len(rec) > 2:
             kernels[name]["sm_mhz_in_kernel"] = round(rec[2])
-    kind, work = kernel_work(dom, wl)
+    kind, work = kernel_work(dom, wl, lr)
     avg_s = dom_prof[dom][0] / dom_prof[dom][1] * 1e-3
     if kind == "tensor":
         achieved = work / avg_s / 1e12
@@ -597,12 +652,13 @@ def main():
 
     cpu = None
     if not args.no_cpu_baseline:
-        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl)
+        lo = lora_np(wl, args) if lr else None
+        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl, lora=lo)
         t0 = time.perf_counter()
-        oracle_step(sample, wl.k, wl.backward, args.router_linear)
+        oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
         dt = time.perf_counter() - t0
         sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
-        cpu = {"value": step_flops(sub_wl) / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        cpu = {"value": step_flops(sub_wl, lr) / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {ts} of {wl.T} tokens, all {wl.E} experts, "
                          f"{'fwd+bwd' if wl.backward else 'fwd'} in float64, one run of {dt:.1f} s"}
 

@@ -225,6 +225,56 @@ int moe_layer_bwd_dw_f32(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16*
                          int accumulate, float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * LoRA adapters on the stacked expert weights.
+ * Source: fused-MoE Triton project summary (sourcepulse), Highlighted
+ * Details: LoRA on the fused expert weights. The pages give no formulas; the
+ * update is the published LoRA form (Hu et al., 2021): a frozen W [out, in]
+ * is used as W + scale * B A. Here one adapter per expert on each stacked
+ * weight, gate|up fused:
+ *   A_gu [E,r,H], B_gu [E,2I,r] on W_gu;  A_d [E,r,I], B_d [E,H,r] on W_d,
+ * all bf16, row-major; r a multiple of 8 in [8, 512]; one scale.
+ * moe_experts_fwd_lora -- moe_experts_fwd with the adapted weights. The low-
+ * rank term is not formed as a matrix: each expert GEMM runs over [act | Z]
+ * and [W | B] along K (its accumulator takes both), where
+ *   Z_gu = scale * Xp A_gu^T  and  Z_d = scale * h A_d^T      [P, r] bf16
+ * are written to the caller's Z_gu / Z_d (outputs, kept for the backward).
+ * Errors: as moe_experts_fwd; r out of range -> MOE_ERR_INVALID_ARG.
+ */
+int moe_experts_fwd_lora(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                         int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, int r,
+                         float scale, const moe_bf16* A_gu, const moe_bf16* B_gu, const moe_bf16* A_d,
+                         const moe_bf16* B_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, moe_bf16* Z_gu,
+                         moe_bf16* Z_d, moe_stream_t stream);
+
+/* Bytes of workspace moe_layer_bwd_lora needs (0 for invalid sizes). */
+size_t moe_layer_bwd_lora_workspace_bytes(int T, int E, int k, int H, int I, int r, int recompute_gu);
+
+/*
+ * moe_layer_bwd_lora -- backward of the adapted layer. With G the gradient
+ * reaching a stacked weight (that of W, equal to that of W + scale B A):
+ *   dA = scale B^T G,  dB = scale G A^T      per expert (chain rule),
+ * computed without forming G: dA_gu = V_gu^T Xp, dB_gu = dGU^T Z_gu,
+ * dA_d = V_d^T (w h), dB_d = dYp^T (w Z_d) over each expert's rows, with
+ * V_d = scale dYp B_d and V_gu = scale dGU B_gu (which also extend the dgrad
+ * GEMMs along K, as in the forward).
+ * dA_gu [E,r,H], dB_gu [E,2I,r], dA_d [E,r,I], dB_d [E,H,r]: fp32 outputs;
+ * accumulate != 0 adds to them (experts without rows add nothing), else
+ * they are overwritten (zeros for such experts).
+ * dW_gu / dW_d: bf16 gradients of the base weights, or NULL to skip them
+ * (frozen base weights: their two GEMMs are not run).
+ * Z_gu, Z_d: the forward's. Every other argument and error as moe_layer_bwd;
+ * ws >= moe_layer_bwd_lora_workspace_bytes(...).
+ */
+int moe_layer_bwd_lora(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                       const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                       const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                       const moe_bf16* W_gu, const moe_bf16* W_d, int r, float scale, const moe_bf16* A_gu,
+                       const moe_bf16* B_gu, const moe_bf16* A_d, const moe_bf16* B_d, const moe_bf16* Z_gu,
+                       const moe_bf16* Z_d, moe_bf16* dX, float* dA_gu, float* dB_gu, float* dA_d, float* dB_d,
+                       int accumulate, moe_bf16* dW_gu, moe_bf16* dW_d, float* dlogits, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/*
  * Gather-fused variants -- the same results as moe_experts_fwd and
  * moe_layer_bwd, reading the activations in token order: the GEMMs load the
  * rows of X [T,H] (and of dY [T,H]) by token index t = sorted_pair[r] / k

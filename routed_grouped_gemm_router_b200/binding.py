@@ -43,6 +43,11 @@ _SIGNATURES = {
                                                                                      _c_size, _c_void]),
     "moe_layer_bwd_x_dw_f32": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 5 + [_c_int, _c_void, _c_void,
                                                                                        _c_size, _c_void]),
+    "moe_experts_fwd_lora": (_c_int, [_c_void] * 4 + [_c_int] * 5 + [_c_void] * 2 + [_c_int, ctypes.c_float]
+                             + [_c_void] * 9 + [_c_void]),
+    "moe_layer_bwd_lora_workspace_bytes": (_c_size, [_c_int] * 7),
+    "moe_layer_bwd_lora": (_c_int, [_c_void] * 10 + [_c_int] * 5 + [_c_void] * 2 + [_c_int, ctypes.c_float]
+                           + [_c_void] * 11 + [_c_int] + [_c_void] * 4 + [_c_size, _c_void]),
     "moe_router_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_router_fwd": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void,
                                 _c_void, _c_void, _c_size, _c_void]),
@@ -177,6 +182,78 @@ def moe_experts_fwd(Xp, offsets, sorted_pair, topk_w, T, E, k, W_gu, W_d, h=None
         _ptr(Xp), _ptr(offsets), _ptr(sorted_pair), _ptr(topk_w), T, E, k, H, I, _ptr(W_gu), _ptr(W_d),
         _ptr(h), _ptr(gu_save), _ptr(O), _stream(stream)))
     return h, gu_save, O
+
+
+def _lora_check(lora, E, H, I):
+    r = lora["A_gu"].shape[1]
+    _need(lora["A_gu"], torch.bfloat16, (E, r, H), "A_gu")
+    _need(lora["B_gu"], torch.bfloat16, (E, 2 * I, r), "B_gu")
+    _need(lora["A_d"], torch.bfloat16, (E, r, I), "A_d")
+    _need(lora["B_d"], torch.bfloat16, (E, H, r), "B_d")
+    return r
+
+
+def moe_experts_fwd_lora(Xp, offsets, sorted_pair, topk_w, T, E, k, W_gu, W_d, lora: dict, h=None, gu_save=None,
+                         O=None, Z_gu=None, Z_d=None, save_gu=True, stream=None):
+    """moe_experts_fwd with LoRA adapters: lora = {A_gu, B_gu, A_d, B_d
+    (bf16), scale}. Returns h, gu_save, O, Z_gu, Z_d (the adapter
+    activations the backward takes)."""
+    P = T * k
+    H = W_gu.shape[2]
+    I = W_d.shape[2]
+    dev = Xp.device
+    _need(Xp, torch.bfloat16, (P, H), "Xp")
+    r = _lora_check(lora, E, H, I)
+    h = torch.empty(P, I, dtype=torch.bfloat16, device=dev) if h is None else h
+    if gu_save is None and save_gu:
+        gu_save = torch.empty(P, 2 * I, dtype=torch.bfloat16, device=dev)
+    O = torch.empty(P, H, dtype=torch.bfloat16, device=dev) if O is None else O
+    Z_gu = torch.empty(P, r, dtype=torch.bfloat16, device=dev) if Z_gu is None else Z_gu
+    Z_d = torch.empty(P, r, dtype=torch.bfloat16, device=dev) if Z_d is None else Z_d
+    _check("moe_experts_fwd_lora", lib().moe_experts_fwd_lora(
+        _ptr(Xp), _ptr(offsets), _ptr(sorted_pair), _ptr(topk_w), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), r,
+        float(lora["scale"]), _ptr(lora["A_gu"]), _ptr(lora["B_gu"]), _ptr(lora["A_d"]), _ptr(lora["B_d"]),
+        _ptr(h), _ptr(gu_save), _ptr(O), _ptr(Z_gu), _ptr(Z_d), _stream(stream)))
+    return h, gu_save, O, Z_gu, Z_d
+
+
+def moe_layer_bwd_lora(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
+                       W_gu, W_d, lora: dict, Z_gu, Z_d, out=None, ws=None, stream=None, accumulate=False,
+                       base_grads=False):
+    """Backward of the adapted layer: dX, dlogits and the fp32 adapter
+    gradients dA_gu, dB_gu, dA_d, dB_d (added to out's when accumulate);
+    base_grads=True also gives the bf16 dW_gu, dW_d (else the base weights
+    are frozen and their GEMMs skipped)."""
+    H = W_gu.shape[2]
+    I = W_d.shape[2]
+    dev = dY.device
+    r = _lora_check(lora, E, H, I)
+    if accumulate and not (out and all(n in out for n in ("dA_gu", "dB_gu", "dA_d", "dB_d"))):
+        raise ValueError("accumulate needs dA_gu, dB_gu, dA_d and dB_d given in `out`")
+    o = dict(out or {})
+    f32 = torch.float32
+    o.setdefault("dX", torch.empty(T, H, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dlogits", torch.empty(T, E, dtype=f32, device=dev))
+    o.setdefault("dA_gu", torch.empty(E, r, H, dtype=f32, device=dev))
+    o.setdefault("dB_gu", torch.empty(E, 2 * I, r, dtype=f32, device=dev))
+    o.setdefault("dA_d", torch.empty(E, r, I, dtype=f32, device=dev))
+    o.setdefault("dB_d", torch.empty(E, H, r, dtype=f32, device=dev))
+    for n, shape in (("dA_gu", (E, r, H)), ("dB_gu", (E, 2 * I, r)), ("dA_d", (E, r, I)), ("dB_d", (E, H, r))):
+        _need(o[n], f32, shape, n)
+    if base_grads:
+        o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev))
+        o.setdefault("dW_d", torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
+    need = lib().moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, r, 1 if gu_save is None else 0)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("moe_layer_bwd_lora", lib().moe_layer_bwd_lora(
+        _ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
+        _ptr(sorted_pair), _ptr(pair_pos), T, E, k, H, I, _ptr(W_gu), _ptr(W_d), r, float(lora["scale"]),
+        _ptr(lora["A_gu"]), _ptr(lora["B_gu"]), _ptr(lora["A_d"]), _ptr(lora["B_d"]), _ptr(Z_gu), _ptr(Z_d),
+        _ptr(o["dX"]), _ptr(o["dA_gu"]), _ptr(o["dB_gu"]), _ptr(o["dA_d"]), _ptr(o["dB_d"]),
+        1 if accumulate else 0, _ptr(o.get("dW_gu") if base_grads else None),
+        _ptr(o.get("dW_d") if base_grads else None), _ptr(o["dlogits"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
 
 
 def moe_combine(O, pair_pos, T, k, Y=None, stream=None):

@@ -147,6 +147,16 @@ struct GemmParams {
   float* out_f32;             // wgrad: fp32 output in place of `out` (NULL: bf16 to `out`), same strides
   int accumulate;             // wgrad with out_f32: out_f32 += acc (fp32 add) instead of out_f32 = acc
   unsigned long long* clock_acc;  // profiling (NULL: off): [0] += SM cycles, [1] += ns of each MMA issuer's loop
+  // K extension (row-grouped kinds): after the ceil(K / 64) K blocks of tmA /
+  // tmB, nkb2 more come from tmA2 / tmB2 into the same accumulator, i.e. the
+  // GEMM of [A | A2] and [B | B2] along K. Same row coordinates as the first
+  // pair, except an MN-major B2, whose K rows are b_rows2 per expert. Used for
+  // the low-rank adapter term (A2 = scale * Z, B2 = the adapter's B or A).
+  CUtensorMap tmA2;
+  CUtensorMap tmB2;
+  int nkb2;
+  int b_rows2;
+  float out_scale;  // FwdDown / BwdDgradGateUp / bf16 wgrad epilogue: out = out_scale * (w *) acc
 };
 
 template <int CG>
@@ -195,7 +205,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     // pair tiles start at 256-row steps; the one-CTA tile is the segment's tail
     ti.row0 = s_off[lo] + (CG == 2 ? ti.m_blk * kBM : ((s_off[lo + 1] - s_off[lo]) / kBM) * kBM);
     ti.rows = s_off[lo + 1] - ti.row0;
-    ti.num_kb = (p.K + kBK - 1) / kBK;
+    ti.num_kb = (p.K + kBK - 1) / kBK + p.nkb2;
   }
   return ti;
 }
@@ -389,6 +399,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
     if constexpr (GATHER != kNoGather) tma_prefetch_desc(&p.tmG);
+    if (p.nkb2 > 0) {
+      tma_prefetch_desc(&p.tmA2);
+      tma_prefetch_desc(&p.tmB2);
+    }
   }
   if (warp == 1) {
     if constexpr (CG == 2) {
@@ -448,11 +462,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       (void)prefetch_only;
       const CUtensorMap* mapA = &p.tmA;
       const CUtensorMap* mapB = &p.tmB;
+      int kb_local = kb;
+      int b_rows = p.b_rows;
       if constexpr (kWgrad) {
         mapA = p.expert_maps + ti.e;
         mapB = p.expert_maps + p.E + ti.e;
+      } else {
+        const int nkb1 = (p.K + kBK - 1) / kBK;
+        if (kb >= nkb1) {  // K extension
+          mapA = &p.tmA2;
+          mapB = &p.tmB2;
+          kb_local = kb - nkb1;
+          b_rows = p.b_rows2;
+        }
       }
-      const int kx = kb * kBK;
+      const int kx = kb_local * kBK;
       const int r = static_cast<int>(rank);
       // box c of B lands 8 KiB (MN-major boxes of 64 x 64) or 16 KiB
       // (K-major boxes of 128 rows) after the previous one
@@ -468,7 +492,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         if constexpr (CG == 1) { nbox_b = 2; b_step_y = kBNc; b_step_bytes = kBTileBytes; }
       } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
         ax = kx; ay = ti.row0 + r * kBMc;
-        bx = ti.n_blk * kBN + r * kBNc; by = ti.e * p.b_rows + kx;
+        bx = ti.n_blk * kBN + r * kBNc; by = ti.e * b_rows + kx;
         nbox_b = CG == 2 ? 2 : 4; b_step_x = 64; b_step_bytes = 8192;
       } else {  // wgrad: K rows are the expert's permuted rows
         ax = ti.m_blk * kBM + r * kBMc; ay = ti.row0 + kx;
@@ -894,7 +918,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           if (kEpiWarps == 4 && tr_q == 0 && r < wrows)
             p.dw_part[(wrow0 + r) * (kDwSlotsPerNTile * p.n_tiles) + kDwSlotsPerNTile * ti.n_blk + 1] = 0.f;
         }
-      } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (w *) acc
+      } else {  // FwdDown (weighted), BwdDgradGateUp, BwdWgrad: plain bf16 store of (scale * w *) acc
+        wq *= p.out_scale;
 #pragma unroll 1
         for (int ch = ch0; ch < ch0 + kChunks; ch += 2) {
           uint32_t a0[32], a1[32];

@@ -18,6 +18,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "grouped_gemm.cuh"
+#include "lora.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 #include "router_bwd.cuh"
@@ -139,6 +140,15 @@ enum ProfSlot : int {
   kProfRouterWgrad,
   kProfRouterSumSplits,
   kProfRouterDgrad,
+  kProfLoraZGateUp,
+  kProfLoraZDown,
+  kProfLoraVDown,
+  kProfLoraVGateUp,
+  kProfLoraWeightRows,
+  kProfLoraDAGateUp,
+  kProfLoraDBGateUp,
+  kProfLoraDADown,
+  kProfLoraDBDown,
   kProfSlots
 };
 const char* const kProfNames[kProfSlots] = {
@@ -147,7 +157,9 @@ const char* const kProfNames[kProfSlots] = {
     "gather_dy",      "gemm_recompute_gate_up", "gemm_bwd_dgrad_down", "gemm_bwd_dgrad_gate_up",
     "combine_dx",     "gemm_bwd_wgrad_gate_up", "gemm_bwd_wgrad_down", "router_bwd",
     "router_split_w", "gemm_router_logits",  "router_split_dlogits",   "gemm_router_wgrad",
-    "router_sum_splits", "gemm_router_dgrad"};
+    "router_sum_splits", "gemm_router_dgrad", "gemm_lora_z_gate_up", "gemm_lora_z_down", "gemm_lora_v_down",
+    "gemm_lora_v_gate_up", "lora_weight_rows", "gemm_lora_da_gate_up", "gemm_lora_db_gate_up", "gemm_lora_da_down",
+    "gemm_lora_db_down"};
 
 struct Profiler {
   std::mutex mu;
@@ -302,7 +314,49 @@ GemmParams base_params(int E, int64_t P, const int32_t* offsets) {
   p.E = E;
   p.P = P;
   p.offsets = offsets;
+  p.out_scale = 1.0f;
   return p;
+}
+
+// ------------------------------------------------------------ LoRA adapters
+// One adapter per expert on each stacked weight: the layer uses
+// W_gu + scale B_gu A_gu and W_d + scale B_d A_d. The forward keeps the
+// adapter activations Z_gu = scale Xp A_gu^T and Z_d = scale h A_d^T [P, r].
+struct LoraArgs {
+  int r = 0;
+  float scale = 1.0f;
+  const moe_bf16* A_gu = nullptr;  // [E, r, H]
+  const moe_bf16* B_gu = nullptr;  // [E, 2I, r]
+  const moe_bf16* A_d = nullptr;   // [E, r, I]
+  const moe_bf16* B_d = nullptr;   // [E, H, r]
+  moe_bf16* Z_gu = nullptr;        // [P, r]
+  moe_bf16* Z_d = nullptr;         // [P, r]
+  float* dA_gu = nullptr;          // backward outputs, fp32
+  float* dB_gu = nullptr;
+  float* dA_d = nullptr;
+  float* dB_d = nullptr;
+  bool accumulate = false;
+};
+constexpr int kLoraMaxRank = 512;
+
+bool lora_rank_ok(int r) { return r >= 8 && r <= kLoraMaxRank && r % 8 == 0; }
+
+// K extension of a row-grouped GEMM by the adapter term: A2 [P, r] (K-major),
+// and B2 either K-major [E * b_rows, r] (forward kinds, the base B's rows) or
+// MN-major [E * r, N] (dgrad kinds: K rows = the adapter rank). Columns of A2
+// past r read as zeros (out of the map), so B2 rows past r multiply zeros.
+bool set_lora_ext(GemmParams& g, const moe_bf16* A2, int64_t P, const moe_bf16* B2, int E, int r, bool b_mn,
+                  int b_rows_or_n) {
+  if (!make_map(&g.tmA2, A2, r, P, 64, 128)) return false;
+  if (b_mn) {
+    if (!make_map(&g.tmB2, B2, b_rows_or_n, static_cast<uint64_t>(E) * r, 64, 64)) return false;
+    g.b_rows2 = r;
+  } else {
+    if (!make_map(&g.tmB2, B2, r, static_cast<uint64_t>(E) * b_rows_or_n, 64, 128)) return false;
+    g.b_rows2 = b_rows_or_n;
+  }
+  g.nkb2 = cdiv(r, kBK);
+  return true;
 }
 
 bool shape_ok(int T, int E, int k) {
@@ -311,10 +365,12 @@ bool shape_ok(int T, int E, int k) {
 bool dims_ok(int H) { return H > 0 && H % 8 == 0; }
 
 struct BwdLayout {
-  size_t dYp, dGU, hw, dXp, dw_part, maps, gu, total;
+  size_t dYp, dGU, hw, dXp, dw_part, maps, gu, V_d, V_gu, Zw_d, total;
 };
 // gather: the GEMMs read dY (and X) rows by token, so there is no dYp copy.
-BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute, bool gather = false) {
+// lora_r > 0: room for the adapter terms V_d, V_gu, w * Z_d [P, r] and the
+// tensor maps of the four adapter-gradient GEMMs.
+BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute, bool gather = false, int lora_r = 0) {
   const size_t P = static_cast<size_t>(T) * k;
   BwdLayout L;
   size_t off = 0;
@@ -323,8 +379,12 @@ BwdLayout bwd_layout(int T, int E, int k, int H, int I, bool recompute, bool gat
   L.hw = off; off += round256(P * I * 2);
   L.dXp = off; off += round256(P * H * 2);
   L.dw_part = off; off += round256(P * kDwSlotsPerNTile * cdiv(I, kBN) * 4);
-  L.maps = off; off += round256(static_cast<size_t>(4) * E * sizeof(CUtensorMap));
+  L.maps = off; off += round256(static_cast<size_t>(lora_r > 0 ? 12 : 4) * E * sizeof(CUtensorMap));
   L.gu = off; off += recompute ? round256(P * 2 * I * 2) : 0;
+  const size_t zr = lora_r > 0 ? round256(P * lora_r * 2) : 0;
+  L.V_d = off; off += zr;
+  L.V_gu = off; off += zr;
+  L.Zw_d = off; off += zr;
   L.total = off;
   return L;
 }
@@ -581,18 +641,49 @@ namespace moe {
 namespace {
 // The two expert GEMMs of the forward. gather: `src` is X [T, H] in token
 // order and the gate/up GEMM gathers its rows; otherwise `src` is Xp [P, H].
+// lora (optional, permuted rows only): the adapted weights W + scale B A,
+// with the adapter activations Z_gu, Z_d written for the backward.
 int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, const int32_t* sorted_pair,
                      const float* topk_w, int T, int E, int k, int H, int I, const moe_bf16* W_gu,
-                     const moe_bf16* W_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, cudaStream_t stream) {
+                     const moe_bf16* W_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, cudaStream_t stream,
+                     const LoraArgs* lora = nullptr) {
   const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
+  if (lora != nullptr && (gather || !lora_rank_ok(lora->r))) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
   if (P == 0) return MOE_OK;
   if (!ok_ptr(Xp) || !ok_ptr(offsets) || !ok_ptr(sorted_pair) || !ok_opt(topk_w) || !ok_ptr(W_gu) ||
       !ok_ptr(W_d) || !ok_ptr(h) || !ok_opt(gu_save) || !ok_ptr(O))
     return MOE_ERR_INVALID_ARG;
+  if (lora != nullptr && (!ok_ptr(lora->A_gu) || !ok_ptr(lora->B_gu) || !ok_ptr(lora->A_d) || !ok_ptr(lora->B_d) ||
+                          !ok_ptr(lora->Z_gu) || !ok_ptr(lora->Z_d)))
+    return MOE_ERR_INVALID_ARG;
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
+  const int tails = tail_ctas(P, E, dev->num_sms);
+
+  // Z = scale * act A^T [P, r]: a plain row-grouped GEMM with N = r whose B
+  // is the adapter's A [E * r, K] (K-major)
+  auto lora_z = [&](const moe_bf16* act, int K, const moe_bf16* A, moe_bf16* Z, int slot) -> int {
+    GemmParams z = base_params(E, P, offsets);
+    if (!make_map(&z.tmA, act, K, P, 64, 128) ||
+        !make_map(&z.tmB, A, K, static_cast<uint64_t>(E) * lora->r, 64, 128))
+      return MOE_ERR_CUDA;
+    z.sorted_pair = sorted_pair;
+    z.N = lora->r;
+    z.K = K;
+    z.I = I;
+    z.b_rows = lora->r;
+    z.n_tiles = cdiv(lora->r, kBN);
+    z.out = Z;
+    z.out_ld = lora->r;
+    z.out_scale = lora->scale;
+    return launch_gemm<kFwdDown>(z, rowgrouped_grid(P, E, z.n_tiles, dev->num_sms), stream, slot, tails,
+                                 dev->num_sms);
+  };
+  if (lora != nullptr) {
+    if (int st = lora_z(Xp, H, lora->A_gu, lora->Z_gu, kProfLoraZGateUp)) return st;
+  }
 
   GemmParams gu = base_params(E, P, offsets);
   if (!make_map(&gu.tmB, W_gu, H, static_cast<uint64_t>(E) * 2 * I, 64, 128)) return MOE_ERR_CUDA;
@@ -611,10 +702,14 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   gu.out = h;
   gu.out_ld = I;
   gu.gu = gu_save;
+  if (lora != nullptr && !set_lora_ext(gu, lora->Z_gu, P, lora->B_gu, E, lora->r, false, 2 * I)) return MOE_ERR_CUDA;
   const int gu_grid = rowgrouped_grid(P, E, gu.n_tiles, dev->num_sms);
   if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(gu, gu_grid, stream, kProfFwdGateUp)
-                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
+                      : launch_gemm<kFwdGateUp>(gu, gu_grid, stream, kProfFwdGateUp, tails, dev->num_sms))
     return st;
+  if (lora != nullptr) {
+    if (int st = lora_z(h, I, lora->A_d, lora->Z_d, kProfLoraZDown)) return st;
+  }
 
   GemmParams dn = base_params(E, P, offsets);
   if (!make_map(&dn.tmA, h, I, P, 64, 128) || !make_map(&dn.tmB, W_d, I, static_cast<uint64_t>(E) * H, 64, 128))
@@ -628,7 +723,9 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   dn.n_tiles = cdiv(H, kBN);
   dn.out = O;
   dn.out_ld = H;
-  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown, tail_ctas(P, E, dev->num_sms), dev->num_sms);
+  if (lora != nullptr && !set_lora_ext(dn, lora->Z_d, P, lora->B_d, E, lora->r, false, H)) return MOE_ERR_CUDA;
+  return launch_gemm<kFwdDown>(dn, rowgrouped_grid(P, E, dn.n_tiles, dev->num_sms), stream, kProfFwdDown, tails,
+                               dev->num_sms);
 }
 }  // namespace
 }  // namespace moe
@@ -667,6 +764,29 @@ size_t moe_layer_bwd_x_workspace_bytes(int T, int E, int k, int H, int I, int re
   return bwd_layout(T, E, k, H, I, recompute_gu != 0, true).total;
 }
 
+size_t moe_layer_bwd_lora_workspace_bytes(int T, int E, int k, int H, int I, int r, int recompute_gu) {
+  if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I) || !lora_rank_ok(r)) return 0;
+  return bwd_layout(T, E, k, H, I, recompute_gu != 0, false, r).total;
+}
+
+int moe_experts_fwd_lora(const moe_bf16* Xp, const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w,
+                         int T, int E, int k, int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, int r,
+                         float scale, const moe_bf16* A_gu, const moe_bf16* B_gu, const moe_bf16* A_d,
+                         const moe_bf16* B_d, moe_bf16* h, moe_bf16* gu_save, moe_bf16* O, moe_bf16* Z_gu,
+                         moe_bf16* Z_d, moe_stream_t stream) {
+  LoraArgs a;
+  a.r = r;
+  a.scale = scale;
+  a.A_gu = A_gu;
+  a.B_gu = B_gu;
+  a.A_d = A_d;
+  a.B_d = B_d;
+  a.Z_gu = Z_gu;
+  a.Z_d = Z_d;
+  return experts_fwd_impl(Xp, false, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, h, gu_save, O, stream,
+                          &a);
+}
+
 }  // extern "C"
 
 namespace moe {
@@ -682,33 +802,54 @@ void set_dw_out(GemmParams& p, void* dW, bool dw_f32, bool accumulate) {
 // otherwise `src` is Xp [P, H] and dY is first gathered into dYp.
 // dw_f32: dW_gu / dW_d are fp32 (the wgrad accumulators unrounded), else
 // bf16; accumulate (fp32 only): dW += the gradient instead of dW = it.
+// lora (optional, permuted rows only): backward of the adapted layer; the
+// adapter gradients go to lora->dA_* / dB_* (fp32), and dW_gu / dW_d may then
+// be NULL (frozen base weights: their GEMMs are skipped).
 int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const moe_bf16* gu_save,
                    const moe_bf16* h, const float* probs, const int32_t* topk_idx, const float* topk_w,
                    const int32_t* offsets, const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k,
                    int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, void* dW_gu, void* dW_d,
-                   bool dw_f32, bool accumulate, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                   bool dw_f32, bool accumulate, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream,
+                   const LoraArgs* lora = nullptr) {
   const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
-  if (!ok_ptr(dW_gu) || !ok_ptr(dW_d) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
+  if (lora != nullptr) {
+    if (gather || !lora_rank_ok(lora->r) || !ok_opt(dW_gu) || !ok_opt(dW_d)) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(lora->A_gu) || !ok_ptr(lora->B_gu) || !ok_ptr(lora->A_d) || !ok_ptr(lora->B_d) ||
+        !ok_ptr(lora->dA_gu) || !ok_ptr(lora->dB_gu) || !ok_ptr(lora->dA_d) || !ok_ptr(lora->dB_d))
+      return MOE_ERR_INVALID_ARG;
+  } else if (!ok_ptr(dW_gu) || !ok_ptr(dW_d)) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
   if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_opt(h) || !ok_ptr(probs) ||
                 !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(sorted_pair) || !ok_ptr(pair_pos) ||
                 !ok_ptr(W_gu) || !ok_ptr(W_d) || !ok_ptr(dX) || !ok_ptr(dlogits)))
     return MOE_ERR_INVALID_ARG;
+  if (P > 0 && lora != nullptr && (!ok_ptr(lora->Z_gu) || !ok_ptr(lora->Z_d))) return MOE_ERR_INVALID_ARG;
   (void)h;  // not read: the dgrad-down epilogue recomputes h = silu(g) * u from g|u
   const bool recompute = (gu_save == nullptr);
-  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute, gather);
+  const int lora_r = lora != nullptr ? lora->r : 0;
+  const BwdLayout L = bwd_layout(T, E, k, H, I, recompute, gather, lora_r);
   if (P > 0 && (ws_bytes < L.total || !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
   const size_t dw_elem = dw_f32 ? 4 : 2;
   const size_t dw_gu_bytes = static_cast<size_t>(E) * 2 * I * H * dw_elem;
   const size_t dw_d_bytes = static_cast<size_t>(E) * H * I * dw_elem;
-  if (P == 0) {  // no rows: every expert is empty, all weight gradients are zero
-    if (accumulate) return MOE_OK;  // dW += 0
-    if (cudaMemsetAsync(dW_gu, 0, dw_gu_bytes, stream) != cudaSuccess ||
-        cudaMemsetAsync(dW_d, 0, dw_d_bytes, stream) != cudaSuccess)
+  if (P == 0) {  // no rows: every expert is empty, all weight gradients are zero (dW += 0 if accumulating)
+    if (!accumulate && ((dW_gu != nullptr && cudaMemsetAsync(dW_gu, 0, dw_gu_bytes, stream) != cudaSuccess) ||
+                        (dW_d != nullptr && cudaMemsetAsync(dW_d, 0, dw_d_bytes, stream) != cudaSuccess)))
       return MOE_ERR_CUDA;
+    if (lora != nullptr && !lora->accumulate) {
+      const size_t r = static_cast<size_t>(lora->r), e = static_cast<size_t>(E);
+      if (cudaMemsetAsync(lora->dA_gu, 0, e * r * H * 4, stream) != cudaSuccess ||
+          cudaMemsetAsync(lora->dB_gu, 0, e * 2 * I * r * 4, stream) != cudaSuccess ||
+          cudaMemsetAsync(lora->dA_d, 0, e * r * I * 4, stream) != cudaSuccess ||
+          cudaMemsetAsync(lora->dB_d, 0, e * H * r * 4, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     return MOE_OK;
   }
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -749,11 +890,37 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     rc.n_tiles = cdiv(I, 128);
     rc.out = nullptr;
     rc.gu = gu_ws;
+    if (lora != nullptr && !set_lora_ext(rc, lora->Z_gu, P, lora->B_gu, E, lora->r, false, 2 * I)) return MOE_ERR_CUDA;
     const int grid = rowgrouped_grid(P, E, rc.n_tiles, dev->num_sms);
     if (int st = gather ? launch_gemm<kFwdGateUp, kGatherA>(rc, grid, stream, kProfRecomputeGateUp)
                         : launch_gemm<kFwdGateUp>(rc, grid, stream, kProfRecomputeGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
     gu = gu_ws;
+  }
+  // Adapter terms of the dgrad GEMMs: V = scale * act B [P, r], a plain
+  // row-grouped GEMM (the dgrad-gate/up kind) whose MN-major B is the
+  // adapter's B [E * K, r]. The dgrads then take [V] and the adapter's A as
+  // their K extension.
+  moe_bf16* V_d = reinterpret_cast<moe_bf16*>(w8 + L.V_d);
+  moe_bf16* V_gu = reinterpret_cast<moe_bf16*>(w8 + L.V_gu);
+  auto lora_v = [&](const moe_bf16* act, int K, const moe_bf16* Bm, moe_bf16* V, int slot) -> int {
+    GemmParams v = base_params(E, P, offsets);
+    if (!make_map(&v.tmA, act, K, P, 64, 128) ||
+        !make_map(&v.tmB, Bm, lora->r, static_cast<uint64_t>(E) * K, 64, 64))
+      return MOE_ERR_CUDA;
+    v.N = lora->r;
+    v.K = K;
+    v.I = I;
+    v.b_rows = K;
+    v.n_tiles = cdiv(lora->r, kBN);
+    v.out = V;
+    v.out_ld = lora->r;
+    v.out_scale = lora->scale;
+    return launch_gemm<kBwdDgradGateUp>(v, rowgrouped_grid(P, E, v.n_tiles, dev->num_sms), stream, slot,
+                                        tail_ctas(P, E, dev->num_sms), dev->num_sms);
+  };
+  if (lora != nullptr) {
+    if (int st = lora_v(dYp, H, lora->B_d, V_d, kProfLoraVDown)) return st;
   }
   // 3. dgrad through down + SwiGLU backward: dGU, hw, partial dw
   {
@@ -777,10 +944,14 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     bd.gu = const_cast<moe_bf16*>(gu);
     bd.hw_out = hw;
     bd.dw_part = dw_part;
+    if (lora != nullptr && !set_lora_ext(bd, V_d, P, lora->A_d, E, lora->r, true, I)) return MOE_ERR_CUDA;
     const int grid = rowgrouped_grid(P, E, bd.n_tiles, dev->num_sms);
     if (int st = gather ? launch_gemm<kBwdDgradDown, kGatherA>(bd, grid, stream, kProfDgradDown)
                         : launch_gemm<kBwdDgradDown>(bd, grid, stream, kProfDgradDown, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
+  }
+  if (lora != nullptr) {
+    if (int st = lora_v(dGU, 2 * I, lora->B_gu, V_gu, kProfLoraVGateUp)) return st;
   }
   // 4. dgrad through gate/up: dXp = dGU W_gu[e]
   {
@@ -795,6 +966,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     bx.n_tiles = cdiv(H, kBN);
     bx.out = dXp;
     bx.out_ld = H;
+    if (lora != nullptr && !set_lora_ext(bx, V_gu, P, lora->A_gu, E, lora->r, true, H)) return MOE_ERR_CUDA;
     if (int st = launch_gemm<kBwdDgradGateUp>(bx, rowgrouped_grid(P, E, bx.n_tiles, dev->num_sms), stream,
                                               kProfDgradGateUp, tail_ctas(P, E, dev->num_sms), dev->num_sms))
       return st;
@@ -807,7 +979,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   // 6. weight gradients, K = the expert's rows. Each launch first writes
   //    per-expert copies of its two tensor maps, clipped at the segment end.
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(w8 + L.maps);
-  {
+  if (dW_gu != nullptr) {
     GemmParams wg = base_params(E, P, offsets);
     if (!make_map(&wg.tmA, dGU, 2 * I, P, 64, 64)) return MOE_ERR_CUDA;
     if (gather) {  // B = X rows by token (its per-expert map copy is unused)
@@ -834,7 +1006,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
                         : launch_gemm<kBwdWgrad>(wg, grid, stream, kProfWgradGateUp))
       return st;
   }
-  {
+  if (dW_d != nullptr) {
     GemmParams wd = base_params(E, P, offsets);
     if (!make_map(&wd.tmB, hw, I, P, 64, 64)) return MOE_ERR_CUDA;
     if (gather) {  // A = dY rows by token (its per-expert map copy is unused)
@@ -860,6 +1032,55 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     if (int st = gather ? launch_gemm<kBwdWgrad, kGatherA>(wd, grid, stream, kProfWgradDown)
                         : launch_gemm<kBwdWgrad>(wd, grid, stream, kProfWgradDown))
       return st;
+  }
+  // 6b. adapter gradients (fp32): per expert over its rows
+  //   dA_gu = V_gu^T Xp, dB_gu = dGU^T Z_gu, dA_d = V_d^T hw, dB_d = dYp^T (w Z_d)
+  // (V, Z carry the scale; hw and w Z_d the routing weight), each a weight-
+  // gradient GEMM with its own per-expert tensor maps.
+  if (lora != nullptr) {
+    const int r = lora->r;
+    moe_bf16* Zw_d = reinterpret_cast<moe_bf16*>(w8 + L.Zw_d);
+    {
+      ProfScope ps(kProfLoraWeightRows, stream);
+      const int64_t n = P * (r / 8);
+      const int blocks = static_cast<int>(cdiv(n, 256) < dev->num_sms * 8 ? cdiv(n, 256) : dev->num_sms * 8);
+      if (launch_pdl(lora_weight_rows_kernel, dim3(blocks), dim3(256), 0, stream,
+                     reinterpret_cast<const uint4*>(lora->Z_d), sorted_pair, topk_w, P, r / 8,
+                     reinterpret_cast<uint4*>(Zw_d)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    struct Wg {
+      const moe_bf16* a;  // [P, M]
+      int M;
+      const moe_bf16* b;  // [P, N]
+      int N;
+      float* out;
+      int slot;
+    };
+    const Wg jobs[4] = {{V_gu, r, Xp, H, lora->dA_gu, kProfLoraDAGateUp},
+                        {dGU, 2 * I, lora->Z_gu, r, lora->dB_gu, kProfLoraDBGateUp},
+                        {V_d, r, hw, I, lora->dA_d, kProfLoraDADown},
+                        {dYp, H, Zw_d, r, lora->dB_d, kProfLoraDBDown}};
+    for (int j = 0; j < 4; ++j) {
+      const Wg& w = jobs[j];
+      GemmParams g = base_params(E, P, offsets);
+      if (!make_map(&g.tmA, w.a, w.M, P, 64, 64) || !make_map(&g.tmB, w.b, w.N, P, 64, 64)) return MOE_ERR_CUDA;
+      CUtensorMap* m = maps + (4 + 2 * j) * E;
+      if (launch_pdl(build_expert_maps_kernel, dim3(cdiv(2 * E, 8)), dim3(256), 0, stream, g.tmA, g.tmB, offsets, E,
+                     m) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      g.expert_maps = m;
+      g.M = w.M;
+      g.N = w.N;
+      g.I = I;
+      g.m_tiles = cdiv(w.M, kBM);
+      g.n_tiles = cdiv(w.N, kBN);
+      g.out_ld = w.N;
+      g.out_expert_stride = static_cast<int64_t>(w.M) * w.N;
+      set_dw_out(g, w.out, true, lora->accumulate);
+      const int64_t tiles = static_cast<int64_t>(E) * g.m_tiles * g.n_tiles;
+      if (int st = launch_gemm<kBwdWgrad>(g, pair_grid(tiles, dev->num_sms), stream, w.slot)) return st;
+    }
   }
   // 7. router logits gradient
   {
@@ -903,6 +1124,32 @@ int moe_layer_bwd_x(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_sa
                     float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return layer_bwd_impl(dY, X, true, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k, H,
                         I, W_gu, W_d, dX, dW_gu, dW_d, false, false, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_layer_bwd_lora(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                       const float* probs, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                       const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k, int H, int I,
+                       const moe_bf16* W_gu, const moe_bf16* W_d, int r, float scale, const moe_bf16* A_gu,
+                       const moe_bf16* B_gu, const moe_bf16* A_d, const moe_bf16* B_d, const moe_bf16* Z_gu,
+                       const moe_bf16* Z_d, moe_bf16* dX, float* dA_gu, float* dB_gu, float* dA_d, float* dB_d,
+                       int accumulate, moe_bf16* dW_gu, moe_bf16* dW_d, float* dlogits, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  LoraArgs a;
+  a.r = r;
+  a.scale = scale;
+  a.A_gu = A_gu;
+  a.B_gu = B_gu;
+  a.A_d = A_d;
+  a.B_d = B_d;
+  a.Z_gu = const_cast<moe_bf16*>(Z_gu);
+  a.Z_d = const_cast<moe_bf16*>(Z_d);
+  a.dA_gu = dA_gu;
+  a.dB_gu = dB_gu;
+  a.dA_d = dA_d;
+  a.dB_d = dB_d;
+  a.accumulate = accumulate != 0;
+  return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
+                        H, I, W_gu, W_d, dX, dW_gu, dW_d, false, false, dlogits, ws, ws_bytes, stream, &a);
 }
 
 int moe_layer_bwd_x_dw_f32(const moe_bf16* dY, const moe_bf16* X, const moe_bf16* gu_save, const moe_bf16* h,

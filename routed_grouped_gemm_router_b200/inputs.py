@@ -124,6 +124,18 @@ def router_logits(X: torch.Tensor, W_r: torch.Tensor, bias: torch.Tensor | None)
     return logits.contiguous()
 
 
+def make_lora(E: int, H: int, I: int, r: int, seed: int = 0, std: float = 0.02) -> dict:
+    """Seeded LoRA adapters for the stacked expert weights, bf16-rounded:
+    A_gu [E, r, H], B_gu [E, 2I, r], A_d [E, r, I], B_d [E, H, r], entries
+    N(0, std) (B nonzero, unlike a fresh adapter, so that the term is
+    exercised)."""
+    g = torch.Generator().manual_seed(seed)
+    return dict(A_gu=(torch.randn(E, r, H, generator=g) * std).to(torch.bfloat16),
+                B_gu=(torch.randn(E, 2 * I, r, generator=g) * std).to(torch.bfloat16),
+                A_d=(torch.randn(E, r, I, generator=g) * std).to(torch.bfloat16),
+                B_d=(torch.randn(E, H, r, generator=g) * std).to(torch.bfloat16))
+
+
 def small_inputs(T, H, E, k, I, seed=0, with_dy=True, zipf_s=0.0, dead=0) -> LayerInputs:
     """Convenience: an ad-hoc problem size (test shapes)."""
     return make_inputs(Workload("adhoc", T, H, E, k, I, zipf_s=zipf_s, dead_experts=dead),

@@ -8,8 +8,10 @@ token index (moe_experts_fwd_x / moe_layer_bwd_x): no Xp / dYp buffers
 slower, so the default keeps the permuted copies.
 ``forward_from_x`` / ``backward_to_x`` also run the router Linear
 (moe_router_fwd in place of moe_route; moe_router_bwd after moe_layer_bwd,
-adding the router's share to dX and giving dW_r). All buffers are torch CUDA
-tensors; nothing here does arithmetic.
+adding the router's share to dX and giving dW_r). ``forward_lora`` /
+``backward_lora`` run the layer with LoRA adapters on the stacked expert
+weights (moe_experts_fwd_lora / moe_layer_bwd_lora). All buffers are torch
+CUDA tensors; nothing here does arithmetic.
 """
 from __future__ import annotations
 
@@ -35,6 +37,9 @@ class LayerState:
     Y: torch.Tensor
     logits: torch.Tensor | None = None
     X: torch.Tensor | None = None  # token-order input, kept for the gather-fused backward
+    lora: dict | None = None       # adapters {A_gu, B_gu, A_d, B_d, scale} of a forward_lora
+    Z_gu: torch.Tensor | None = None  # scale * Xp A_gu^T [P, r]
+    Z_d: torch.Tensor | None = None   # scale * h A_d^T [P, r]
 
 
 def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
@@ -70,6 +75,35 @@ def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, g
     return LayerState(T, E, k, idx, w, probs, perm, h, gu, O, Y, X=X if gather else None)
 
 
+def forward_lora(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int, lora: dict,
+                 save_gu: bool = True, bufs: dict | None = None, stream=None) -> LayerState:
+    """``forward`` with the adapted weights W + scale B A (lora = {A_gu [E,r,H],
+    B_gu [E,2I,r], A_d [E,r,I], B_d [E,H,r] bf16, scale})."""
+    b = bufs or {}
+    T, E = logits.shape
+    idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
+    perm = B.moe_permute(idx, E, X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
+    h, gu, O, Z_gu, Z_d = B.moe_experts_fwd_lora(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k, W_gu,
+                                                 W_d, lora, h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"),
+                                                 Z_gu=b.get("Z_gu"), Z_d=b.get("Z_d"), save_gu=save_gu,
+                                                 stream=stream)
+    Y = B.moe_combine(O, perm["pair_pos"], T, k, Y=b.get("Y"), stream=stream)
+    return LayerState(T, E, k, idx, w, probs, perm, h, gu, O, Y, lora=lora, Z_gu=Z_gu, Z_d=Z_d)
+
+
+def backward_lora(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, bufs: dict | None = None,
+                  stream=None, accumulate: bool = False, base_grads: bool = False) -> dict:
+    """dX, dlogits and the fp32 adapter gradients dA_gu, dB_gu, dA_d, dB_d
+    (accumulate=True adds them to the buffers in bufs["grads"]); the base
+    weights are frozen unless base_grads=True."""
+    b = bufs or {}
+    p = st.perm
+    return B.moe_layer_bwd_lora(dY, p["Xp"], st.gu, st.h, st.probs, st.topk_idx, st.topk_w, p["offsets"],
+                                p["sorted_pair"], p["pair_pos"], st.T, st.E, st.k, W_gu, W_d, st.lora, st.Z_gu,
+                                st.Z_d, out=b.get("grads"), ws=b.get("bwd_ws"), stream=stream,
+                                accumulate=accumulate, base_grads=base_grads)
+
+
 def backward(st: LayerState, dY: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, bufs: dict | None = None,
              stream=None, accumulate: bool = False) -> dict:
     """dX, dW_gu, dW_d, dlogits for upstream gradient dY. The weight
@@ -100,9 +134,11 @@ def backward_to_x(st: LayerState, dY: torch.Tensor, X: torch.Tensor, W_r: torch.
 
 
 def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = True, router: bool = False,
-             gather: bool = False, dw_f32: bool = False) -> dict:
+             gather: bool = False, dw_f32: bool = False, lora_r: int = 0) -> dict:
     """Every output and workspace of one forward+backward, allocated once;
-    dw_f32: fp32 weight-gradient buffers."""
+    dw_f32: fp32 weight-gradient buffers; lora_r > 0: the buffers of
+    forward_lora / backward_lora with adapters of rank lora_r (frozen base
+    weights: no dW buffers)."""
     P = T * k
     bf = torch.bfloat16
     dwt = torch.float32 if dw_f32 else bf
@@ -129,6 +165,19 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
     )
     if not gather:
         d["perm"]["Xp"] = torch.empty(P, H, dtype=bf, device=device)
+    if lora_r > 0:
+        r = lora_r
+        f32 = torch.float32
+        d["Z_gu"] = torch.empty(P, r, dtype=bf, device=device)
+        d["Z_d"] = torch.empty(P, r, dtype=bf, device=device)
+        g = d["grads"]
+        del g["dW_gu"], g["dW_d"]
+        g.update(dA_gu=torch.empty(E, r, H, dtype=f32, device=device),
+                 dB_gu=torch.empty(E, 2 * I, r, dtype=f32, device=device),
+                 dA_d=torch.empty(E, r, I, dtype=f32, device=device),
+                 dB_d=torch.empty(E, H, r, dtype=f32, device=device))
+        d["bwd_ws"] = torch.empty(max(lib.moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, r, 0 if save_gu else 1),
+                                      1), dtype=torch.uint8, device=device)
     if router:
         d["logits"] = torch.empty(T, E, dtype=torch.float32, device=device)
         d["dW_r"] = torch.empty(E, H, dtype=torch.float32, device=device)

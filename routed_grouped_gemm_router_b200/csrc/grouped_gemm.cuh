@@ -157,6 +157,15 @@ struct GemmParams {
   int nkb2;
   int b_rows2;
   float out_scale;  // FwdDown / BwdDgradGateUp / bf16 wgrad epilogue: out = out_scale * (w *) acc
+  // Narrow tiles for skinny products (FwdDown, BwdDgradGateUp, wgrad kinds):
+  // bn = 64 (K-major B only) or 128 output columns per tile instead of 256;
+  // the MMA's N shrinks with it, so a product with few columns does not pay
+  // for 256. 0: 256.
+  int bn;
+  // wgrad with out_f32: store the tile transposed, out_f32[e][n][m] (ld =
+  // out_ld = M), so that a product with few rows can be computed as its
+  // transpose with the few rows as narrow columns.
+  int out_transposed;
 };
 
 template <int CG>
@@ -353,6 +362,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   constexpr bool kAMN = kWgrad;
   constexpr bool kBMN = (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || kWgrad);
   constexpr uint32_t kIdesc = idesc_bf16_f32(CG == 2 ? kBM : kBMc, kBN, kAMN, kBMN);
+  constexpr bool kNarrowOk = (KIND == kFwdDown || KIND == kBwdDgradGateUp || KIND == kBwdWgrad) && GATHER == kNoGather;
+  // tile width along N: every coordinate below uses it; the TMEM buffers and
+  // the staged B rows keep their 256-column size (the MMA reads the first bn)
+  const int bn = (kNarrowOk && p.bn > 0) ? p.bn : kBN;
+  const uint32_t idesc = bn == kBN ? kIdesc : idesc_bf16_f32(CG == 2 ? kBM : kBMc, bn, kAMN, kBMN);
+  // B bytes each CTA stages per K block: its bn/2 (pair) or bn columns only
+  // (a K-major B map's box is bn/2 rows high; MN-major boxes are 64 columns)
+  const int b_bytes_cta = KIND == kFwdGateUp ? Cfg::kBBytes : (CG == 2 ? bn / 2 : bn) * kBK * 2;
+  const uint32_t stage_tx = static_cast<uint32_t>(CG * (kATileBytes + b_bytes_cta));
   constexpr uint32_t kALbo = kAMN ? 8192u : 16u;
   constexpr uint32_t kBLbo = kBMN ? 8192u : 16u;
   constexpr uint32_t kAStep = kAMN ? 2048u : 32u;  // bytes per UMMA_K step
@@ -488,17 +506,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         if constexpr (CG == 1) { nbox_b = 2; b_step_y = p.I; b_step_bytes = kBTileBytes; }
       } else if constexpr (KIND == kFwdDown) {
         ax = kx; ay = ti.row0 + r * kBMc;
-        bx = kx; by = ti.e * p.b_rows + ti.n_blk * kBN + r * kBNc;
-        if constexpr (CG == 1) { nbox_b = 2; b_step_y = kBNc; b_step_bytes = kBTileBytes; }
+        bx = kx; by = ti.e * p.b_rows + ti.n_blk * bn + r * (bn / 2);
+        if constexpr (CG == 1) { nbox_b = 2; b_step_y = bn / 2; b_step_bytes = (bn / 2) * kBK * 2; }
       } else if constexpr (KIND == kBwdDgradDown || KIND == kBwdDgradGateUp) {
         ax = kx; ay = ti.row0 + r * kBMc;
-        bx = ti.n_blk * kBN + r * kBNc; by = ti.e * b_rows + kx;
-        nbox_b = CG == 2 ? 2 : 4; b_step_x = 64; b_step_bytes = 8192;
+        bx = ti.n_blk * bn + r * (bn / 2); by = ti.e * b_rows + kx;
+        nbox_b = (CG == 2 ? bn / 2 : bn) / 64; b_step_x = 64; b_step_bytes = 8192;
       } else {  // wgrad: K rows are the expert's permuted rows
         ax = ti.m_blk * kBM + r * kBMc; ay = ti.row0 + kx;
-        bx = ti.n_blk * kBN + r * kBNc; by = ay;
+        bx = ti.n_blk * bn + r * (bn / 2); by = ay;
         nbox_a = 2;
-        nbox_b = 2; b_step_x = 64; b_step_bytes = 8192;
+        nbox_b = (bn / 2) / 64; b_step_x = 64; b_step_bytes = 8192;
       }
       if constexpr (GATHER != kGatherA) {
         for (int c = 0; c < nbox_a; ++c) {
@@ -532,7 +550,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             *s_abort = 1;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], CG * Cfg::kStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
           issue(ti, kb, false, sA + stage * kATileBytes, sB + stage * Cfg::kBBytes,
                 CG == 2 ? mapa_shared(smem_u32(&full_bar[stage]), 0) : 0u, &full_bar[stage]);
           ++issued;
@@ -709,8 +727,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
               const uint64_t adesc = sdesc_sw128(a_addr + kk * kAStep, kALbo, 1024);
               const uint64_t bdesc = sdesc_sw128(b_addr + kk * kBStep, kBLbo, 1024);
-              if constexpr (CG == 2) umma_bf16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-              else umma_bf16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              if constexpr (CG == 2) umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              else umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             if constexpr (CG == 2) {
               umma_commit_pair(smem_u32(&empty_bar[stage]));
@@ -785,8 +803,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       if constexpr (kWgrad) {
         if (ti.num_kb == 0) {  // expert without rows: its weight gradient is zero (unchanged if accumulating)
           if (out_f32 != nullptr && p.accumulate) continue;
-          for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
-            const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
+          for (int ch = ch0; ch < ch0 + kChunks && ch * 32 < bn; ++ch) {
+            const int col = ti.n_blk * bn + ch * 32 + tr_q * 8;
+            if (p.out_transposed && out_f32 != nullptr) {  // rows of the transposed tile: columns here
+              if (lane < wrows) {
+                for (int j = 0; j < 32 && ti.n_blk * bn + ch * 32 + j < p.N; ++j)
+                  out_f32[static_cast<int64_t>(ti.n_blk * bn + ch * 32 + j) * p.out_ld + wrow0 + lane] = 0.f;
+              }
+              continue;
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = i * 8 + tr_row;
@@ -926,22 +951,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           tmem_ld_32x32b_x32(taddr + ch * 32, a0);
           tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, a1);
           tmem_ld_wait();
-          const int col0 = ti.n_blk * kBN + ch * 32;
+          const int col0 = ti.n_blk * bn + ch * 32;
+          const bool in0 = ch * 32 < bn && col0 < p.N;              // warp-uniform
+          const bool in1 = (ch + 1) * 32 < bn && col0 + 32 < p.N;
           if (kWgrad && out_f32 != nullptr) {  // fp32 weight gradient: the accumulator unrounded
             const bool accum = p.accumulate != 0;
-            if (col0 < p.N)
-              emit_chunk_f32(stg, a0, out_f32, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane, accum);
-            if (col0 + 32 < p.N)
+            if (p.out_transposed) {
+              // thread = tile row m; for each column n the warp's 32 rows are
+              // 32 consecutive floats of out[n][.]: 128-byte stores
+              float* col_base = out_f32 + wrow0 + lane;
+              if (lane < wrows && in0) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (col0 + j < p.N) {
+                    float* dst = col_base + static_cast<int64_t>(col0 + j) * p.out_ld;
+                    float v = __uint_as_float(a0[j]);
+                    if (accum) v += *dst;
+                    *dst = v;
+                  }
+                }
+              }
+              if (lane < wrows && in1) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (col0 + 32 + j < p.N) {
+                    float* dst = col_base + static_cast<int64_t>(col0 + 32 + j) * p.out_ld;
+                    float v = __uint_as_float(a1[j]);
+                    if (accum) v += *dst;
+                    *dst = v;
+                  }
+                }
+              }
+              continue;
+            }
+            if (in0) emit_chunk_f32(stg, a0, out_f32, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane, accum);
+            if (in1)
               emit_chunk_f32(stg, a1, out_f32, wrow0, p.out_ld, col0 + 32, p.N, wrows, tr_row, tr_q, lane, accum);
             continue;
           }
           float v[32];
-          if (col0 < p.N) {  // warp-uniform
+          if (in0) {  // warp-uniform
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a0[j]);
             emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0, p.N, wrows, tr_row, tr_q, lane);
           }
-          if (col0 + 32 < p.N) {
+          if (in1) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a1[j]);
             emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0 + 32, p.N, wrows, tr_row, tr_q, lane);

@@ -341,6 +341,15 @@ constexpr int kLoraMaxRank = 512;
 
 bool lora_rank_ok(int r) { return r >= 8 && r <= kLoraMaxRank && r % 8 == 0; }
 
+// Tile width for a product with n output columns: the narrowest of 64
+// (K-major B only: its rows are the columns), 128 and 256 that holds them.
+// An MN-major B keeps at least 128 (64 per CTA, a whole 128-byte swizzle row).
+int narrow_bn(int n, bool b_mn) {
+  if (n <= 64 && !b_mn) return 64;
+  if (n <= 128) return 128;
+  return kBN;
+}
+
 // K extension of a row-grouped GEMM by the adapter term: A2 [P, r] (K-major),
 // and B2 either K-major [E * b_rows, r] (forward kinds, the base B's rows) or
 // MN-major [E * r, N] (dgrad kinds: K rows = the adapter rank). Columns of A2
@@ -666,15 +675,17 @@ int experts_fwd_impl(const moe_bf16* src, bool gather, const int32_t* offsets, c
   // is the adapter's A [E * r, K] (K-major)
   auto lora_z = [&](const moe_bf16* act, int K, const moe_bf16* A, moe_bf16* Z, int slot) -> int {
     GemmParams z = base_params(E, P, offsets);
+    z.bn = narrow_bn(lora->r, false);
+    // K-major B box: bn / 2 rows, the columns each CTA of a pair computes
     if (!make_map(&z.tmA, act, K, P, 64, 128) ||
-        !make_map(&z.tmB, A, K, static_cast<uint64_t>(E) * lora->r, 64, 128))
+        !make_map(&z.tmB, A, K, static_cast<uint64_t>(E) * lora->r, 64, static_cast<uint32_t>(z.bn / 2)))
       return MOE_ERR_CUDA;
     z.sorted_pair = sorted_pair;
     z.N = lora->r;
     z.K = K;
     z.I = I;
     z.b_rows = lora->r;
-    z.n_tiles = cdiv(lora->r, kBN);
+    z.n_tiles = cdiv(lora->r, z.bn);
     z.out = Z;
     z.out_ld = lora->r;
     z.out_scale = lora->scale;
@@ -912,7 +923,8 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     v.K = K;
     v.I = I;
     v.b_rows = K;
-    v.n_tiles = cdiv(lora->r, kBN);
+    v.bn = narrow_bn(lora->r, true);
+    v.n_tiles = cdiv(lora->r, v.bn);
     v.out = V;
     v.out_ld = lora->r;
     v.out_scale = lora->scale;
@@ -1049,6 +1061,8 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
                      reinterpret_cast<uint4*>(Zw_d)) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
+    // Each is computed with the rank as its N (narrow tiles): dA as its
+    // transpose (Xp^T V_gu, hw^T V_d) stored transposed into [r, K].
     struct Wg {
       const moe_bf16* a;  // [P, M]
       int M;
@@ -1056,11 +1070,12 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
       int N;
       float* out;
       int slot;
+      bool transposed;
     };
-    const Wg jobs[4] = {{V_gu, r, Xp, H, lora->dA_gu, kProfLoraDAGateUp},
-                        {dGU, 2 * I, lora->Z_gu, r, lora->dB_gu, kProfLoraDBGateUp},
-                        {V_d, r, hw, I, lora->dA_d, kProfLoraDADown},
-                        {dYp, H, Zw_d, r, lora->dB_d, kProfLoraDBDown}};
+    const Wg jobs[4] = {{Xp, H, V_gu, r, lora->dA_gu, kProfLoraDAGateUp, true},
+                        {dGU, 2 * I, lora->Z_gu, r, lora->dB_gu, kProfLoraDBGateUp, false},
+                        {hw, I, V_d, r, lora->dA_d, kProfLoraDADown, true},
+                        {dYp, H, Zw_d, r, lora->dB_d, kProfLoraDBDown, false}};
     for (int j = 0; j < 4; ++j) {
       const Wg& w = jobs[j];
       GemmParams g = base_params(E, P, offsets);
@@ -1073,9 +1088,11 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
       g.M = w.M;
       g.N = w.N;
       g.I = I;
+      g.bn = narrow_bn(w.N, true);
       g.m_tiles = cdiv(w.M, kBM);
-      g.n_tiles = cdiv(w.N, kBN);
-      g.out_ld = w.N;
+      g.n_tiles = cdiv(w.N, g.bn);
+      g.out_transposed = w.transposed ? 1 : 0;
+      g.out_ld = w.transposed ? w.M : w.N;
       g.out_expert_stride = static_cast<int64_t>(w.M) * w.N;
       set_dw_out(g, w.out, true, lora->accumulate);
       const int64_t tiles = static_cast<int64_t>(E) * g.m_tiles * g.n_tiles;

@@ -431,54 +431,44 @@ bool router_shape_ok(int T, int H, int E) {
 int router_residency(int bn, int stages) {
   const size_t per = rg_smem_bytes(bn, stages) + 1024;  // + the per-CTA reservation
   int r = static_cast<int>((228 * 1024) / per);
-  const int tmem = 512 / rg_tmem_cols(bn);
+  const int tmem = 512 / (2 * rg_tmem_cols(bn));  // two accumulator buffers per CTA
   if (r > tmem) r = tmem;
   return r < 1 ? 1 : r;
 }
 
-// Split-K count: enough units for every resident CTA slot of the device, at
-// most `cap`, never more splits than K blocks.
+// Split-K count: about kRouterUnitsPerCta units for every resident CTA slot
+// of the (persistent) device grid, at most `cap`, never more splits than K
+// blocks.
+#ifndef MOE_ROUTER_UNITS_PER_CTA
+#define MOE_ROUTER_UNITS_PER_CTA 4
+#endif
+constexpr int kRouterUnitsPerCta = MOE_ROUTER_UNITS_PER_CTA;
 int router_splits(int64_t tiles, int k_blocks, int cap, int slots) {
-  int64_t s = (slots + tiles - 1) / tiles;
+  const int64_t want = static_cast<int64_t>(slots) * kRouterUnitsPerCta;
+  int64_t s = (want + tiles - 1) / tiles;
   if (s > cap) s = cap;
   if (s > k_blocks) s = k_blocks;
   return s < 1 ? 1 : static_cast<int>(s);
 }
 
+// Persistent grid: every resident CTA slot of the device, no more than the
+// units.
 template <int KIND>
-int launch_router_gemm(const RouterGemmParams& p, cudaStream_t s, int slot) {
+int launch_router_gemm(const RouterGemmParams& p, cudaStream_t s, int slot, int num_sms) {
   const size_t smem = rg_smem_bytes(p.bn, p.stages);
   if (cudaFuncSetAttribute(router_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
   ProfScope ps(slot, s);
-  const int64_t grid = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.splits;
+  const int64_t units = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.splits;
+  const int64_t slots = static_cast<int64_t>(num_sms) * router_residency(p.bn, p.stages);
+  const int64_t grid = units < slots ? units : slots;
   if (launch_pdl(router_gemm_kernel<KIND>, dim3(static_cast<unsigned>(grid)), dim3(kRgThreads), smem, s, p) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_status();
 }
 
-// Logits + routing in one launch (clusters of two CTAs per 128-token tile).
-// Off by default: measured slower than split-K logits + the routing kernel
-// (77 vs 48 us on T 8192, H 2048, E 128, k 8): the routing epilogue, one
-// thread per token over four warps, takes about 43 us.
-#ifndef MOE_ROUTER_FUSED_ROUTE
-#define MOE_ROUTER_FUSED_ROUTE 0
-#endif
-constexpr bool kRouterFusedRoute = MOE_ROUTER_FUSED_ROUTE != 0;
-template <int KMAX>
-int launch_router_route(const RouterGemmParams& p, cudaStream_t s) {
-  const size_t smem = rg_smem_bytes(p.bn, p.stages, p.N);
-  if (cudaFuncSetAttribute(router_gemm_kernel<kRgLogitsRoute, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  ProfScope ps(kProfRouterLogits, s);
-  if (launch_pdl_clustered(router_gemm_kernel<kRgLogitsRoute, KMAX>, dim3(2 * p.m_tiles), dim3(kRgThreads), smem, s,
-                           2u, p) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return launch_status();
-}
 
 int launch_split3(const float* src, int64_t rows, int cols, int src_ld, int dst_ld, int64_t term_rows,
                   uint16_t* dst, int num_sms, cudaStream_t s, int slot) {
@@ -1204,7 +1194,7 @@ int moe_router_fwd(const moe_bf16* X, const float* W_r, int T, int H, int E, int
   p.M = T;
   p.N = E;
   p.bn = E < 256 ? round_up(E, 16) : 256;
-  p.stages = p.bn <= 128 ? 3 : 4;
+  p.stages = kRgMaxStages;
   p.m_tiles = cdiv(T, kRgBM);
   p.n_tiles = cdiv(E, p.bn);
   p.nkb = cdiv(H, kRgBK);
@@ -1217,21 +1207,7 @@ int moe_router_fwd(const moe_bf16* X, const float* W_r, int T, int H, int E, int
   p.out_split_stride = int64_t(T) * E8;
   if (!make_map(&p.tmA, X, H, T, 64, kRgBM) || !make_map(&p.tmB, w3, H, 3 * int64_t(E), 64, p.bn))
     return MOE_ERR_CUDA;
-  if (E <= kRgRouteMaxE && k <= 32 && kRouterFusedRoute) {
-    // one kernel: K split over the two CTAs of a cluster, routing in the epilogue
-    p.splits = 2;
-    p.n_tiles = 1;
-    p.stages = 4;
-    p.k = k;
-    p.topk_idx = topk_idx;
-    p.topk_w = topk_w;
-    p.probs = probs;
-    p.logits = logits;
-    if (k <= 8) return launch_router_route<8>(p, stream);
-    if (k <= 16) return launch_router_route<16>(p, stream);
-    return launch_router_route<32>(p, stream);
-  }
-  if (int st = launch_router_gemm<kRgLogits>(p, stream, kProfRouterLogits)) return st;
+  if (int st = launch_router_gemm<kRgLogits>(p, stream, kProfRouterLogits, dev->num_sms)) return st;
   ProfScope ps(kProfRoute, stream);
   if (launch_route(nullptr, T, E, k, topk_idx, topk_w, probs, stream, part, p.splits, E8, int64_t(T) * E8, logits) !=
       cudaSuccess)
@@ -1268,7 +1244,7 @@ int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, in
     p.M = H;
     p.N = E;
     p.bn = E < 256 ? round_up(E, 64) : 256;
-    p.stages = p.bn <= 128 ? 3 : 4;
+    p.stages = kRgMaxStages;
     p.m_tiles = cdiv(H, kRgBM);
     p.n_tiles = cdiv(E, p.bn);
     p.nkb = cdiv(T, kRgBK);
@@ -1281,7 +1257,7 @@ int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, in
     p.out_split_stride = int64_t(E) * H;
     if (!make_map(&p.tmA, X, H, T, 64, 64) || !make_map(&p.tmB, dl3, E, 3 * int64_t(T), 64, 64, E8))
       return MOE_ERR_CUDA;
-    if (int st = launch_router_gemm<kRgWgrad>(p, stream, kProfRouterWgrad)) return st;
+    if (int st = launch_router_gemm<kRgWgrad>(p, stream, kProfRouterWgrad, dev->num_sms)) return st;
     if (p.splits > 1) {
       const int64_t n = int64_t(E) * H;
       int64_t blocks = (n / 4 + 255) / 256;
@@ -1300,7 +1276,7 @@ int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, in
     p.M = T;
     p.N = H;
     p.bn = kRgDgradBN;
-    p.stages = 3;
+    p.stages = kRgMaxStages;
     p.m_tiles = cdiv(T, kRgBM);
     p.n_tiles = cdiv(H, p.bn);
     p.nkb = cdiv(E, kRgBK);
@@ -1312,7 +1288,7 @@ int moe_router_bwd(const float* dlogits, const moe_bf16* X, const float* W_r, in
     p.dx_ld = H;
     if (!make_map(&p.tmA, dl3, E, 3 * int64_t(T), 64, kRgBM, E8) || !make_map(&p.tmB, w3, H, 3 * int64_t(E), 64, 64))
       return MOE_ERR_CUDA;
-    if (int st = launch_router_gemm<kRgDgrad>(p, stream, kProfRouterDgrad)) return st;
+    if (int st = launch_router_gemm<kRgDgrad>(p, stream, kProfRouterDgrad, dev->num_sms)) return st;
   }
   return MOE_OK;
 }

@@ -38,7 +38,11 @@ def _run(inp, k, lora, accumulate_onto=None, base_grads=False, save_gu=True):
 
 
 CASES = [(600, 256, 16, 4, 192, 16, 0), (333, 200, 12, 3, 72, 8, 3), (257, 128, 8, 2, 96, 64, 0),
-         (130, 64, 5, 2, 40, 72, 0), (700, 320, 13, 3, 136, 24, 2), (1, 64, 4, 2, 32, 8, 0)]
+         (130, 64, 5, 2, 40, 72, 0), (700, 320, 13, 3, 136, 24, 2), (1, 64, 4, 2, 32, 8, 0),
+         # the largest rank (8 extension K blocks; 256-wide tiles, two N tiles in every skinny product)
+         (300, 128, 40, 4, 64, 512, 0),
+         # sizes that are not multiples of 64 (as in gpt-oss, H = I = 2880), rank 128
+         (420, 288, 9, 3, 288, 128, 0)]
 
 
 @pytest.mark.parametrize("shape", CASES, ids=lambda s: "T%d_H%d_E%d_k%d_I%d_r%d_dead%d" % s)

@@ -110,3 +110,38 @@ def test_router_linear_arguments_rejected_without_device():
     assert lib.moe_router_bwd(p, p, NULL, 16, 16, 4, NULL, p, p, need, NULL) == 1      # dX needs W_r
     assert lib.moe_router_bwd(p, p, p, 16, 16, 4, p, p, p, need - 1, NULL) == 3
     assert "gemm_router_logits" in B.profile_kernel_names()
+
+
+def test_lora_arguments_rejected_without_device():
+    lib = B.lib()
+    p = ctypes.c_void_p(256)
+    odd = ctypes.c_void_p(264 + 2)
+    T, E, k, H, I = 4, 8, 2, 16, 16
+    assert lib.moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, 16, 0) > lib.moe_layer_bwd_workspace_bytes(
+        T, E, k, H, I, 0), "room for the adapter terms"
+    for r in (0, 7, 12, 520):
+        assert lib.moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, r, 0) == 0, f"rank {r}"
+    assert lib.moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, 512, 0) > 0
+
+    def fwd(r=16, a_gu=p, z_gu=p, scale=2.0):
+        # Xp, offsets, sorted_pair, topk_w, T, E, k, H, I, W_gu, W_d, r, scale, A_gu, B_gu, A_d, B_d, h, gu, O, Z_gu, Z_d
+        return lib.moe_experts_fwd_lora(p, p, p, p, T, E, k, H, I, p, p, r, scale, a_gu, p, p, p, p, p, p, z_gu, p,
+                                        NULL)
+
+    assert fwd(r=12) == 1
+    assert fwd(r=520) == 1
+    assert fwd(a_gu=NULL) == 1
+    assert fwd(a_gu=odd) == 1
+    assert fwd(z_gu=NULL) == 1
+    need = lib.moe_layer_bwd_lora_workspace_bytes(T, E, k, H, I, 16, 0)
+
+    def bwd(r=16, da=p, ws_bytes=need, dW_gu=NULL):
+        head = [p] * 10 + [T, E, k, H, I] + [p, p, r, 2.0] + [p] * 4 + [p, p] + [p, da, p, p, p]
+        return lib.moe_layer_bwd_lora(*head, 0, dW_gu, NULL, p, p, ws_bytes, NULL)
+
+    assert bwd(r=9) == 1
+    assert bwd(da=NULL) == 1                 # adapter gradients are required
+    assert bwd(dW_gu=odd) == 1               # an optional base gradient must still be aligned
+    assert bwd(ws_bytes=need - 1) == 3
+    names = B.profile_kernel_names()
+    assert {"gemm_lora_z_gate_up", "gemm_lora_da_down", "lora_weight_rows"} <= set(names)

@@ -194,14 +194,28 @@ Profiler g_prof;
 // A static device array: profiling allocates no device memory.
 __device__ unsigned long long g_gemm_clock[kProfSlots][2];
 
+// Device address of g_gemm_clock on the current device, looked up once per
+// device (NULL if the lookup fails).
+unsigned long long* gemm_clock_base() {
+  constexpr int kMaxDevices = 64;
+  static unsigned long long* base[kMaxDevices] = {};
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return nullptr;
+  if (base[d] == nullptr) {
+    void* b = nullptr;
+    if (cudaGetSymbolAddress(&b, g_gemm_clock) != cudaSuccess) return nullptr;
+    base[d] = static_cast<unsigned long long*>(b);
+  }
+  return base[d];
+}
+
 // Device address of the slot's clock counters when that slot is being
 // profiled, else NULL (the kernels then skip the accounting).
 unsigned long long* gemm_clock_slot(int slot) {
   std::lock_guard<std::mutex> lock(g_prof.mu);
   if (!g_prof.on || (g_prof.only >= 0 && g_prof.only != slot)) return nullptr;
-  void* base = nullptr;
-  if (cudaGetSymbolAddress(&base, g_gemm_clock) != cudaSuccess) return nullptr;
-  return static_cast<unsigned long long*>(base) + 2 * slot;
+  unsigned long long* base = gemm_clock_base();
+  return base != nullptr ? base + 2 * slot : nullptr;
 }
 
 // Brackets one kernel launch with events on its stream when profiling is on.
@@ -1307,9 +1321,8 @@ int moe_profile_enable(int on) {
   g_prof.on = (on != 0);
   g_prof.only = -1;
   if (on) {
-    void* base = nullptr;
-    if (cudaGetSymbolAddress(&base, g_gemm_clock) != cudaSuccess ||
-        cudaMemset(base, 0, sizeof(unsigned long long) * 2 * kProfSlots) != cudaSuccess)
+    unsigned long long* base = gemm_clock_base();
+    if (base == nullptr || cudaMemset(base, 0, sizeof(unsigned long long) * 2 * kProfSlots) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   return MOE_OK;

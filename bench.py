@@ -647,6 +647,11 @@ def main():
             # NVML's reading is a coarse average: the kernel's own counters
             # give the clock it really ran at in the headline pass
             clocks["dominant_gemm_sm_mhz_in_kernel"] = round(dom_prof[dom][2])
+            clocks["note"] = ("in-kernel SM clock = the dominant GEMM's own clock64 cycles / globaltimer ns over its "
+                              "main loops; it sits below NVML's reading because the 1000 W power limit slows the "
+                              "clock inside the tensor-bound kernels, which NVML's coarse sampling does not resolve "
+                              "(the cuBLAS sustained peak in MEASURED_PEAKS.json was taken at a 1327 MHz median with "
+                              "no throttle reason flagged either); no clock lock is set")
     roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name), "algorithmic_per_launch": work,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 

@@ -50,7 +50,6 @@ def kernel_work(name, wl, lora_r=0):
         # term as r more K columns ([act | Z] [W | B])
         "gemm_fwd_gate_up": 4.0 * H * I * P + 4.0 * I * r * P, "gemm_fwd_down": 2.0 * H * I * P + 2.0 * H * r * P,
         "gemm_recompute_gate_up": 4.0 * H * I * P + 4.0 * I * r * P,
-        "gemm_bwd_dgrad_down": 2.0 * H * I * P + 2.0 * I * r * P,
         "gemm_bwd_dgrad_gate_up": 4.0 * H * I * P + 2.0 * H * r * P,
         "gemm_bwd_wgrad_gate_up": 4.0 * H * I * P, "gemm_bwd_wgrad_down": 2.0 * H * I * P,
         # adapter products (useful flops; their tiles are 256 wide in r)
@@ -74,6 +73,11 @@ def kernel_work(name, wl, lora_r=0):
         "gemm_router_wgrad": T * H * 2 + T * E * 4 + E * H * 4, "router_sum_splits": 2 * E * H * 4,
         "gemm_router_dgrad": T * E * 4 + E * H * 4 + 2 * T * H * 2,
         "lora_weight_rows": 2 * P * r * 2 + P * 8,
+        # dgrad through down is HBM-bound by its roofline (these bytes at the
+        # measured copy bandwidth take longer than its flops at the bf16 peak):
+        # dYp, W_d and g|u read; dGU, w*h and the routing-weight partials written
+        "gemm_bwd_dgrad_down": (P * H * 2 + E * H * I * 2 + P * 2 * I * 2 + P * 2 * I * 2 + P * I * 2
+                                + P * 2 * ((I + 255) // 256) * 4 + (P * r * 2 + E * r * I * 2 if r else 0)),
     }
     return "hbm", float(nbytes.get(name, 0))
 

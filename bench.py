@@ -656,7 +656,11 @@ def main():
                               "clock inside the tensor-bound kernels, which NVML's coarse sampling does not resolve "
                               "(the cuBLAS sustained peak in MEASURED_PEAKS.json was taken at a 1327 MHz median with "
                               "no throttle reason flagged either); no clock lock is set")
-    roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name), "algorithmic_per_launch": work,
+    # the committed captures are of the default layer: LoRA, fp32 weight
+    # gradients and gathered operands change what the GEMMs move
+    same_kernels = not (lr or args.dw_f32 or gf)
+    roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name) if same_kernels else None,
+                 "algorithmic_per_launch": work,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 
     cpu = None

@@ -1,6 +1,7 @@
 """The C-ABI library builds, loads without a GPU, exports every function the
 header declares, and rejects bad arguments before touching a device."""
 import ctypes
+import os
 
 import pytest
 
@@ -145,3 +146,46 @@ def test_lora_arguments_rejected_without_device():
     assert bwd(ws_bytes=need - 1) == 3
     names = B.profile_kernel_names()
     assert {"gemm_lora_z_gate_up", "gemm_lora_da_down", "lora_weight_rows"} <= set(names)
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  /* calls that need no device: status strings, workspace sizes, argument checks */
+  if (strcmp(moe_status_str(MOE_OK), moe_status_str(MOE_ERR_INVALID_ARG)) == 0) return 10;
+  if (moe_permute_workspace_bytes(8192, 128, 8) == 0) return 11;
+  if (moe_layer_bwd_workspace_bytes(8192, 128, 8, 2048, 768, 0) == 0) return 12;
+  if (moe_layer_bwd_workspace_bytes(8192, 128, 8, 2047, 768, 0) != 0) return 13;
+  if (moe_layer_bwd_lora_workspace_bytes(8192, 128, 8, 2048, 768, 12, 0) != 0) return 14;
+  if (moe_router_workspace_bytes(8192, 2048, 128) == 0) return 15;
+  void* p = (void*)(size_t)256;
+  if (moe_route((const float*)p, 4, 3, 4, (int32_t*)p, (float*)p, (float*)p, NULL) != MOE_ERR_INVALID_ARG) return 16;
+  if (moe_combine((const moe_bf16*)p, (const int32_t*)p, 4, 2, 12, (moe_bf16*)p, NULL) != MOE_ERR_INVALID_ARG) return 17;
+  if (moe_profile_kernel_name(0) == NULL) return 18;
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+def test_header_is_c_and_matches_the_library(tmp_path):
+    """A plain C99 program compiled against include/moe.h and linked to the
+    built library: the header is valid C, and its declarations resolve to the
+    library's exports and behave as documented without a device."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = B.lib()._name
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, str(src), lib,
+                        f"-Wl,-rpath,{os.path.dirname(lib)}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)

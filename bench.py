@@ -412,22 +412,26 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    def run_fwd(X_, logits_, b):
+        """The layer's forward through the public API."""
+        if rl:
+            return layer.forward_from_x(X_, W_r, W_gu, W_d, wl.k, bufs=b, gather=gf)
+        if lr:
+            return layer.forward_lora(logits_, X_, W_gu, W_d, wl.k, lora, bufs=b)
+        return layer.forward(logits_, X_, W_gu, W_d, wl.k, bufs=b, gather=gf)
+
+    def run_bwd(st, dY_, X_, b):
+        """The layer's backward through the public API."""
+        if rl:
+            return layer.backward_to_x(st, dY_, X_, W_r, W_gu, W_d, bufs=b)
+        if lr:
+            return layer.backward_lora(st, dY_, W_gu, W_d, bufs=b)
+        return layer.backward(st, dY_, W_gu, W_d, bufs=b)
+
     def run_step(X_, logits_, dY_, b):
         """One forward (+ backward) through the public API; (state, grads)."""
-        g = None
-        if rl:
-            st = layer.forward_from_x(X_, W_r, W_gu, W_d, wl.k, bufs=b, gather=gf)
-            if wl.backward:
-                g = layer.backward_to_x(st, dY_, X_, W_r, W_gu, W_d, bufs=b)
-        elif lr:
-            st = layer.forward_lora(logits_, X_, W_gu, W_d, wl.k, lora, bufs=b)
-            if wl.backward:
-                g = layer.backward_lora(st, dY_, W_gu, W_d, bufs=b)
-        else:
-            st = layer.forward(logits_, X_, W_gu, W_d, wl.k, bufs=b, gather=gf)
-            if wl.backward:
-                g = layer.backward(st, dY_, W_gu, W_d, bufs=b)
-        return st, g
+        st = run_fwd(X_, logits_, b)
+        return st, (run_bwd(st, dY_, X_, b) if wl.backward else None)
 
     def step():
         run_step(X, logits, dY, bufs)
@@ -530,7 +534,9 @@ def main():
     # its inputs (X, logits, dY) from pinned host memory and reads its results
     # (Y, dX, dlogits) back. Inputs and outputs are double-buffered and the
     # copies run on two copy streams, so step i+1's upload and step i's
-    # download overlap step i's compute, as a training loop would prefetch.
+    # download overlap step i's compute, as a training loop would prefetch:
+    # the forward starts once X and the logits are in (dY lands meanwhile),
+    # and Y goes back while the backward runs.
     e2e_ms, h2d, d2h = None, 0, 0
     if not args.no_e2e:
         pin = dict(X=inp.X.pin_memory(), logits=inp.logits.pin_memory(),
@@ -554,7 +560,8 @@ def main():
             obufs.append(o)
         up, down = torch.cuda.Stream(), torch.cuda.Stream()
         ev = lambda: torch.cuda.Event()
-        ev_in, ev_used, ev_out, ev_copied = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        ev_in_f, ev_in_b, ev_used = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        ev_y, ev_out, ev_copied = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
         def upload(b):
             with torch.cuda.stream(up):
@@ -562,9 +569,10 @@ def main():
                 din[b]["X"].copy_(pin["X"], non_blocking=True)
                 if not rl:
                     din[b]["logits"].copy_(pin["logits"], non_blocking=True)
+                ev_in_f[b].record(up)  # what the forward reads
                 if wl.backward:
                     din[b]["dY"].copy_(pin["dY"], non_blocking=True)
-                ev_in[b].record(up)
+                ev_in_b[b].record(up)
 
         def run_e2e(nsteps):
             for b in range(2):
@@ -575,14 +583,21 @@ def main():
                 b = i % 2
                 if i + 1 < nsteps:
                     upload((i + 1) % 2)
-                stream.wait_event(ev_in[b])
-                stream.wait_event(ev_copied[b])
-                st, g = run_step(din[b]["X"], din[b]["logits"], din[b]["dY"], obufs[b])
+                stream.wait_event(ev_in_f[b])
+                stream.wait_event(ev_copied[b])  # this buffer's previous results are home
+                st = run_fwd(din[b]["X"], din[b]["logits"], obufs[b])
+                ev_y[b].record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(ev_y[b])
+                    out_h["Y"].copy_(st.Y, non_blocking=True)
+                g = None
+                if wl.backward:
+                    stream.wait_event(ev_in_b[b])
+                    g = run_bwd(st, din[b]["dY"], din[b]["X"], obufs[b])
                 ev_used[b].record(stream)
                 ev_out[b].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_out[b])
-                    out_h["Y"].copy_(st.Y, non_blocking=True)
                     if wl.backward:
                         out_h["dX"].copy_(g["dX"], non_blocking=True)
                         out_h["dlogits"].copy_(g["dlogits"], non_blocking=True)

@@ -294,13 +294,17 @@ inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
 // rest are small), one CTA for one tile time each; the full tiles cost two
 // CTAs each (P / 256 of them). When the average segment is 128 rows or less
 // nearly every tile is a tail.
+#ifndef MOE_TAIL_WEIGHT
+#define MOE_TAIL_WEIGHT 0.65
+#endif
+constexpr double kTailWeight = MOE_TAIL_WEIGHT;
 inline int tail_ctas(int64_t P, int E, int num_sms) {
   if (!kTailTiles || P == 0) return 0;
   int c;
   if (P <= static_cast<int64_t>(128) * E) {
     c = num_sms - 4;
   } else {
-    const double tail = 0.65 * E, full = 2.0 * static_cast<double>(P) / kBM;
+    const double tail = kTailWeight * E, full = 2.0 * static_cast<double>(P) / kBM;
     c = static_cast<int>(num_sms * tail / (tail + full) + 0.5);
   }
   c &= ~1;

@@ -701,8 +701,9 @@ def main():
         "e2e": None if e2e_ms is None else {
             "value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": e2e_ms / args.steps,
-            "note": "pinned host buffers; uploads/downloads on two copy streams overlap compute; "
-                    "no L2 flush (per-step working set >> L2)"},
+            "note": "pinned host buffers; uploads/downloads on two copy streams overlap compute (the forward "
+                    "starts once X and the logits are in, Y goes back during the backward); no L2 flush "
+                    "(per-step working set >> L2)"},
         "gpu_launches": launches, "clocks": clocks, "kernels": kernels,
         "kernels_note": "value, ms_per_step and the roofline kernel come from the first timed pass (events "
                         "around the dominant kernel only); the per-kernel table from a second pass that records "

@@ -3,15 +3,16 @@
 
 One step = the whole layer: moe_route -> moe_permute -> moe_experts_fwd ->
 moe_combine -> moe_layer_bwd on one synthetic batch already resident in HBM.
-Prints ONE JSON line (rank 0). Default workload: the Qwen3-30B-A3B-shaped
-layer (T=8192, H=2048, E=128, k=8, I=768), forward and backward.
+Prints ONE JSON line (rank 0). Default workload: the Qwen3-235B-A22B-shaped
+layer (T=16384, H=4096, E=128, k=8, I=1536), forward and backward.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
-With N > 1 (launched by torch.distributed.run) every rank runs its own
-replica on its own batch (weak scaling, no data-path collective); the time is
-the max over ranks.
+With N > 1 (launched by torch.distributed.run) every rank runs the layer on
+its own batch (weak scaling) and the ranks' weight gradients are summed over
+NCCL after every backward (--grad-sync allreduce | reduce_scatter | none); the
+time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -122,17 +123,33 @@ def kernel_source_sha(kernel=None):
 
 def measured_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary of the same kernel
-    source; None when there is none or the sources changed since."""
+    source, and the summary's file name; (None, None) when there is none or
+    the sources changed since.
+
+    A summary of the workload itself is used as it stands. A summary of a
+    scaled case (fewer experts and tokens, the same rows per expert and the
+    same H, I, k) names the workload it stands for (`scales_to:`) and the
+    ratio of units processed (`scale_factor:`, full-size pairs over the
+    case's pairs); its per-launch traffic is multiplied by that ratio, since
+    every operand the kernel moves (expert weights, expert rows) grows in
+    proportion to the experts and pairs."""
     sha = kernel_source_sha(kernel)
-    for p in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
+    direct, scaled = None, None
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.txt"))):
         text = open(p).read()
-        if (re.search(rf"^kernel: {re.escape(kernel)}$", text, re.M)
-                and re.search(rf"^workload: {re.escape(workload)}$", text, re.M)
+        if not (re.search(rf"^kernel: {re.escape(kernel)}$", text, re.M)
                 and re.search(rf"^source_sha: {sha}$", text, re.M)):
-            m = re.search(r"^traffic_bytes_per_launch: ([0-9.eE+]+)$", text, re.M)
-            if m:
-                return float(m.group(1))
-    return None
+            continue
+        m = re.search(r"^traffic_bytes_per_launch: ([0-9.eE+]+)$", text, re.M)
+        if not m:
+            continue
+        if re.search(rf"^workload: {re.escape(workload)}$", text, re.M):
+            direct = (float(m.group(1)), os.path.basename(p))
+        elif re.search(rf"^scales_to: {re.escape(workload)}$", text, re.M):
+            f = re.search(r"^scale_factor: ([0-9.eE+]+)$", text, re.M)
+            if f:
+                scaled = (float(m.group(1)) * float(f.group(1)), os.path.basename(p) + f" (x{f.group(1)})")
+    return direct or scaled or (None, None)
 
 
 class ClockSampler:
@@ -229,27 +246,49 @@ def oracle_step(inp_sub, k, backward, router=False, lora=None):
             orc.router_logits_backward(bwd["dlogits"], inp_sub.X, inp_sub.W_r)
 
 
+CPU_SAMPLE_EXPERTS = 16
+
+
 def cpu_sample(inp, wl, target_s, router=False, lora=None):
-    """The first T_s tokens of the batch (all E experts), T_s sized so one
-    oracle fwd+bwd takes about target_s seconds on the host cores."""
+    """A bounded sample of the batch for the oracle: the first T_s tokens
+    routed over the first E_s = min(E, 16) experts (the logits, router weight
+    and expert weights cut to those experts), T_s sized so one oracle step
+    takes about target_s seconds on the host cores. The oracle widens every
+    expert weight it is given to float64 on each call, so the expert cut keeps
+    that fixed cost (and the host memory) bounded on the large layers; the
+    per-expert problem (H, I, k) is the workload's own. Returns the sample,
+    T_s, E_s and the sample's adapters (or None)."""
     import copy
+
+    es = min(wl.E, max(CPU_SAMPLE_EXPERTS, 2 * wl.k))
+    lo = None
+    if lora is not None:
+        lo = {n: (v[:es] if n != "scale" else v) for n, v in lora.items()}
 
     def sub(ts):
         s = copy.copy(inp)
-        s.X, s.logits = inp.X[:ts].contiguous(), inp.logits[:ts].contiguous()
+        s.X = inp.X[:ts].contiguous()
+        s.logits = inp.logits[:ts, :es].contiguous()
+        s.W_r = inp.W_r[:es].contiguous()
+        s.W_gu, s.W_d = inp.W_gu[:es].contiguous(), inp.W_d[:es].contiguous()
         s.dY = inp.dY[:ts].contiguous() if inp.dY is not None else None
         return s
 
     ts = min(wl.T, 64)
     t0 = time.perf_counter()
-    oracle_step(sub(ts), wl.k, wl.backward, router, lora)
+    oracle_step(sub(ts), wl.k, wl.backward, router, lo)
     dt = time.perf_counter() - t0
     while ts < wl.T and dt < target_s / 4:
         ts = min(wl.T, ts * 4)
         t0 = time.perf_counter()
-        oracle_step(sub(ts), wl.k, wl.backward, router, lora)
+        oracle_step(sub(ts), wl.k, wl.backward, router, lo)
         dt = time.perf_counter() - t0
-    return sub(ts), ts
+    return sub(ts), ts, es, lo
+
+
+def sample_desc(wl, ts, es):
+    return (f"first {ts} of {wl.T} tokens routed over the first {es} of {wl.E} experts (logits and weights cut "
+            f"to them), {'fwd+bwd' if wl.backward else 'fwd'} in float64")
 
 
 def step_flops(wl, lora_r=0):
@@ -305,8 +344,8 @@ def run_reference(args, wl, rank):
         return
     inp = make_inputs(wl, seed=args.seed)
     lo = lora_np(wl, args) if args.lora else None
-    sample, ts = cpu_sample(inp, wl, target_s=args.ref_step_s, router=args.router_linear, lora=lo)
-    sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
+    sample, ts, es, lo = cpu_sample(inp, wl, target_s=args.ref_step_s, router=args.router_linear, lora=lo)
+    sub_wl = type(wl)(wl.name, ts, wl.H, es, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
     for _ in range(args.warmup):
         oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
     t0 = time.perf_counter()
@@ -314,7 +353,7 @@ def run_reference(args, wl, rank):
         oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
     dt = (time.perf_counter() - t0) / args.steps
     value = step_flops(sub_wl, args.lora) / dt / 1e12
-    desc = f"first {ts} of {wl.T} tokens, all {wl.E} experts, {'fwd+bwd' if wl.backward else 'fwd'} in float64"
+    desc = sample_desc(wl, ts, es)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
@@ -340,7 +379,10 @@ def workload_config(wl, args):
             "lora_rank": int(getattr(args, "lora", 0)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
-            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+            "parallelism": (f"dp{args.gpus} (own batch per rank, weight gradients summed over NCCL: "
+                            f"{getattr(args, 'grad_sync', 'allreduce')})" if args.gpus > 1 and wl.backward
+                            and getattr(args, "grad_sync", "allreduce") != "none"
+                            else f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU")}
 
 
 def main():
@@ -348,7 +390,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qwen3-30b-a3b", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="qwen3-235b-a22b", choices=sorted(WORKLOADS))
     ap.add_argument("--forward-only", action="store_true")
     ap.add_argument("--cuda-graph", action="store_true",
                     help="capture one whole step in a CUDA graph after warm-up and time its replays")
@@ -360,21 +402,30 @@ def main():
                     help="weight gradients written as fp32 (the wgrad accumulators unrounded) instead of bf16")
     ap.add_argument("--router-linear", action="store_true",
                     help="include the router Linear (logits = X W_r^T and its backward) in the step")
+    ap.add_argument("--grad-sync", default="allreduce", choices=["allreduce", "reduce_scatter", "none"],
+                    help="N > 1: how the ranks' weight gradients are summed after each backward (NCCL)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling cases)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (scaled profiling cases: fewer experts, the same rows per expert with --tokens)")
+    ap.add_argument("--sustained-s", type=float, default=2.0,
+                    help="length of the back-to-back sustained pass reported beside the headline (0: skip)")
     ap.add_argument("--cpu-target-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
-    if args.forward_only or args.tokens:
+    if args.forward_only or args.tokens or args.experts:
         T = args.tokens or wl.T
-        name = wl.name if T == wl.T else f"{wl.name}-t{T}"
-        wl = type(wl)(name, T, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts,
+        E = args.experts or wl.E
+        if E < wl.k:
+            ap.error("--experts must be at least the workload's top-k")
+        name = wl.name + (f"-e{E}" if E != wl.E else "") + (f"-t{T}" if T != wl.T else "")
+        wl = type(wl)(name, T, wl.H, E, wl.k, wl.I, wl.zipf_s, min(wl.dead_experts, E - wl.k),
                       wl.backward and not args.forward_only)
 
     world, rank, local_rank = world_info()
@@ -412,6 +463,35 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    # Data parallel (N > 1): the weight gradients live in one flat buffer and
+    # are summed over the ranks after every backward (one NCCL collective),
+    # timed on its own with events around it.
+    grad_flat, grad_extra, sync_evs = None, [], []
+    sync = world > 1 and wl.backward and args.grad_sync != "none"
+    if sync and args.cuda_graph:
+        ap.error("--cuda-graph captures one rank's step; the N > 1 step with its gradient exchange runs eagerly")
+    if sync:
+        from routed_grouped_gemm_router_b200 import dp
+        g = bufs["grads"]
+        names = [n for n in ("dW_gu", "dW_d", "dA_gu", "dB_gu", "dA_d", "dB_d") if n in g]
+        grad_flat, views = dp.flat_views({n: tuple(g[n].shape) for n in names}, g[names[0]].dtype, dev)
+        g.update(views)
+        if rl:
+            grad_extra = [bufs["dW_r"]]
+
+    def exchange():
+        """Sums the weight gradients over the ranks (N > 1)."""
+        if not sync:
+            return
+        if torch.cuda.is_current_stream_capturing():
+            dp.sync_weight_grads(grad_flat, extra=grad_extra, op=args.grad_sync)
+            return
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dp.sync_weight_grads(grad_flat, extra=grad_extra, op=args.grad_sync)
+        b.record(stream)
+        sync_evs.append((a, b))
+
     def run_fwd(X_, logits_, b):
         """The layer's forward through the public API."""
         if rl:
@@ -429,9 +509,14 @@ def main():
         return layer.backward(st, dY_, W_gu, W_d, bufs=b)
 
     def run_step(X_, logits_, dY_, b):
-        """One forward (+ backward) through the public API; (state, grads)."""
+        """One forward (+ backward and, with N > 1, the weight-gradient
+        exchange) through the public API; (state, grads)."""
         st = run_fwd(X_, logits_, b)
-        return st, (run_bwd(st, dY_, X_, b) if wl.backward else None)
+        g = None
+        if wl.backward:
+            g = run_bwd(st, dY_, X_, b)
+            exchange()
+        return st, g
 
     def step():
         run_step(X, logits, dY, bufs)
@@ -468,13 +553,14 @@ def main():
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
-    def timed_steps(only=None, profile=True, replay=False):
-        """K steps, each bracketed by events on the launching stream, L2
-        flushed between steps outside the events; the library also records
-        CUDA events around its kernel launches (all of them, or only kernel
-        `only`)."""
+    def timed_steps(only=None, profile=True, replay=False, nsteps=None):
+        """K (or nsteps) steps, each bracketed by events on the launching
+        stream, L2 flushed between steps outside the events; the library also
+        records CUDA events around its kernel launches (all of them, or only
+        kernel `only`)."""
+        nsteps = nsteps or args.steps
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+               for _ in range(nsteps)]
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -482,7 +568,7 @@ def main():
             B.profile_enable(True)
             if only is not None:
                 B.profile_only(only)
-        for i in range(args.steps):
+        for i in range(nsteps):
             flush.zero_()
             evs[i][0].record(stream)
             if replay:
@@ -517,6 +603,7 @@ def main():
     # library events inside it) and the dominant kernel is timed in an extra
     # eager pass right after.
     dom = warm_dominant
+    sync_evs.clear()
     if sampler:
         sampler.window(True)
     if graph is not None:
@@ -525,10 +612,21 @@ def main():
         step_ms, dom_prof = timed_steps(only=dom)
     if sampler:
         sampler.window(False)
+    torch.cuda.synchronize()
+    sync_ms = sum(a.elapsed_time(b) for a, b in sync_evs)  # the exchange inside the headline steps
     if graph is not None:
         _, dom_prof = timed_steps(only=dom)
     total_ms = sum(step_ms)
     prof_step_ms, prof = timed_steps()
+    # Pass 3, sustained: the same steps back to back for about --sustained-s
+    # seconds with no library events (a training run's steady state under the
+    # power limit), reported beside the headline.
+    sus_ms = None
+    if args.sustained_s > 0:
+        n_sus = max(args.steps, int(args.sustained_s * 1e3 / (total_ms / args.steps)) + 1)
+        if world > 1:  # every rank runs the same number of steps
+            n_sus = int(max_over_ranks([n_sus], dev)[0])
+        sus_ms, _ = timed_steps(profile=False, replay=graph is not None, nsteps=n_sus)
 
     # End to end through the public API with host buffers: every step copies
     # its inputs (X, logits, dY) from pinned host memory and reads its results
@@ -594,6 +692,7 @@ def main():
                 if wl.backward:
                     stream.wait_event(ev_in_b[b])
                     g = run_bwd(st, din[b]["dY"], din[b]["X"], obufs[b])
+                    exchange()
                 ev_used[b].record(stream)
                 ev_out[b].record(stream)
                 with torch.cuda.stream(down):
@@ -619,9 +718,11 @@ def main():
         e2e_ms = e0.elapsed_time(e1)
     clocks = sampler.stop() if sampler else None
 
+    sus_total = sum(sus_ms) if sus_ms else None
     if world > 1:
-        t_max, e_max = max_over_ranks([total_ms, e2e_ms or 0.0], dev)
+        t_max, e_max, s_max, sync_ms = max_over_ranks([total_ms, e2e_ms or 0.0, sus_total or 0.0, sync_ms], dev)
         total_ms, e2e_ms = t_max, (e_max if e2e_ms is not None else None)
+        sus_total = s_max if sus_ms else None
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -674,21 +775,21 @@ def main():
     # the committed captures are of the default layer: LoRA, fp32 weight
     # gradients and gathered operands change what the GEMMs move
     same_kernels = not (lr or args.dw_f32 or gf)
-    roof.update({"kernel": dom, "traffic": measured_traffic(dom, wl.name) if same_kernels else None,
+    traffic, traffic_src = measured_traffic(dom, wl.name) if same_kernels else (None, None)
+    roof.update({"kernel": dom, "traffic": traffic, "traffic_source": traffic_src,
                  "algorithmic_per_launch": work,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 
     cpu = None
     if not args.no_cpu_baseline:
         lo = lora_np(wl, args) if lr else None
-        sample, ts = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl, lora=lo)
+        sample, ts, es, lo = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl, lora=lo)
         t0 = time.perf_counter()
         oracle_step(sample, wl.k, wl.backward, args.router_linear, lo)
         dt = time.perf_counter() - t0
-        sub_wl = type(wl)(wl.name, ts, wl.H, wl.E, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
+        sub_wl = type(wl)(wl.name, ts, wl.H, es, wl.k, wl.I, wl.zipf_s, wl.dead_experts, wl.backward)
         cpu = {"value": step_flops(sub_wl, lr) / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"first {ts} of {wl.T} tokens, all {wl.E} experts, "
-                         f"{'fwd+bwd' if wl.backward else 'fwd'} in float64, one run of {dt:.1f} s"}
+               "sample": sample_desc(wl, ts, es) + f", one run of {dt:.1f} s"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -709,6 +810,20 @@ def main():
                         "around the dominant kernel only); the per-kernel table from a second pass that records "
                         "every launch (serialised, and later under the power limit)",
         "ms_per_step_profiled": sum(prof_step_ms) / args.steps,
+        "grad_sync": None if not sync else {
+            "op": args.grad_sync, "backend": "nccl",
+            "bytes_per_step": grad_flat.numel() * grad_flat.element_size() + sum(t.numel() * t.element_size()
+                                                                                  for t in grad_extra),
+            "ms_per_step": sync_ms / args.steps,
+            "note": "sum of the ranks' weight gradients after each backward, inside the timed step; events "
+                    "around the collective in the headline pass, max over ranks"},
+        "sustained": None if not sus_ms else {
+            "value": aggregate_tflops(world, flops, len(sus_ms), sus_total), "unit": UNIT,
+            "ms_per_step": sus_total / len(sus_ms), "steps": len(sus_ms), "seconds": sus_total * 1e-3,
+            "pct_of_bf16_peak_sustained": aggregate_tflops(world, flops, len(sus_ms), sus_total) / world
+            / peaks["bf16_tflops_sustained"],
+            "note": "the same steps back to back after the per-kernel pass, no library events; L2 flushed "
+                    "between steps outside the events"},
     }
     print(json.dumps(line), flush=True)
     if world > 1:

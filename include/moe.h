@@ -128,7 +128,10 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
  * 4,194,304 pairs); larger problems return MOE_ERR_WORKSPACE and launch
  * nothing. The first call on a device looks up that array's device address
  * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. All calls share the array: calls whose executions
+ * any stream capture. The address is kept for the life of the process: after
+ * cudaDeviceReset (or anything else that destroys and re-creates the device's
+ * context) it is stale, so do not call this entry point again in that
+ * process. All calls share the array: calls whose executions
  * overlap on the GPU (other streams or host threads on the same device) race
  * on it. Leftover contents from earlier calls are harmless: every value read
  * is written earlier in the same call.
@@ -213,8 +216,8 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
  * dW_gu / dW_d 16-byte aligned, contiguous. Every other argument, the
  * workspace (moe_layer_bwd_workspace_bytes) and the error codes are those
  * of moe_layer_bwd.
- * Source: "Optimizing Mixture of Experts Models" (axolotl issue #3155),
- * expert weights [num_experts, 2*intermediate_dim, hidden_dim] and
+ * Source: "[MoE] Improve moe kernels for unsloth fine tuning #3812", the
+ * stacked expert weights [num_experts, 2*intermediate_dim, hidden_dim] and
  * [num_experts, hidden_dim, intermediate_dim]; the pages train in bf16 and
  * leave the gradient's precision open.
  */
@@ -278,8 +281,9 @@ int moe_layer_bwd_lora(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* g
  * Gather-fused variants -- the same results as moe_experts_fwd and
  * moe_layer_bwd, reading the activations in token order: the GEMMs load the
  * rows of X [T,H] (and of dY [T,H]) by token index t = sorted_pair[r] / k
- * with 16-byte asynchronous copies issued by the GEMM itself, so no permuted
- * copies Xp / dYp are made or read.
+ * with row-gather TMA loads (tile::gather4, four 128-byte row pieces per
+ * load) issued by the GEMM itself, so no permuted copies Xp / dYp are made
+ * or read.
  * Source: fused-MoE Triton project summary (sourcepulse), How It Works:
  * inputs are sorted by expert for coalesced grouped-GEMM reads; here the
  * sort is applied inside the GEMM's operand loads. moe_permute may then be

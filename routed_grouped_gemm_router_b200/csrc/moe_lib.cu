@@ -195,12 +195,15 @@ Profiler g_prof;
 __device__ unsigned long long g_gemm_clock[kProfSlots][2];
 
 // Device address of g_gemm_clock on the current device, looked up once per
-// device (NULL if the lookup fails).
+// device (NULL if the lookup fails); the cache is guarded by its own mutex so
+// host threads may call in concurrently.
 unsigned long long* gemm_clock_base() {
   constexpr int kMaxDevices = 64;
   static unsigned long long* base[kMaxDevices] = {};
+  static std::mutex mu;
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (base[d] == nullptr) {
     void* b = nullptr;
     if (cudaGetSymbolAddress(&b, g_gemm_clock) != cudaSuccess) return nullptr;

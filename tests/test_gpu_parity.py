@@ -23,7 +23,7 @@ SHAPES = [
     (96, 128, 16, 1, 128),     # k = 1 (weight = 1)
     (1, 64, 4, 2, 64),         # a single token
     (3, 72, 5, 2, 40),         # fewer rows than one tile, tiny tails
-    (1200, 512, 32, 4, 384),   # several M tiles per expert
+    (1200, 512, 32, 4, 384),   # 32 experts of about 150 rows (one pair tile or a tail each)
 ]
 
 
@@ -47,6 +47,34 @@ def test_layer_matches_oracle(shape):
     U.assert_rel(U.to_np(grads["dW_gu"]), bwd["dW_gu"], "dW_gu")
     U.assert_rel(U.to_np(grads["dW_d"]), bwd["dW_d"], "dW_d")
     U.assert_rel(U.to_np(grads["dlogits"]), bwd["dlogits"], "dlogits")
+
+
+def test_one_expert_spans_many_pair_tiles():
+    """Expert 0 is in every token's top-k: its segment is 2148 rows, eight
+    256-row pair tiles and a 100-row tail (the one-CTA tail tiles); the other
+    three experts share the second slot (about 716 rows each: two pair tiles
+    and a tail of more than 128 rows). Every stored intermediate (g, u, h, O)
+    and every output and gradient element by element against the oracle."""
+    T, H, E, k, I = 2148, 256, 4, 2, 320
+    inp = small_inputs(T, H, E, k, I, seed=11)
+    logits = inp.logits.clone()
+    logits[:, 0] += 30.0
+    inp.logits = logits.contiguous()
+    st, grads = U.run_layer(inp, k)
+    fwd, bwd = U.oracle_full(inp, k)
+    U.check_routing_exact(st, fwd)
+    assert fwd["counts"][0] == T and fwd["counts"][1:].min() > 512 + 128
+    U.assert_rel(U.to_np(st.gu)[:, :I], fwd["g"], "g")
+    U.assert_rel(U.to_np(st.gu)[:, I:], fwd["u"], "u")
+    U.assert_rel(U.to_np(st.h), fwd["h"], "h")
+    U.assert_rel(U.to_np(st.O), fwd["O"], "O")
+    U.assert_rel(U.to_np(st.Y), fwd["Y"], "Y")
+    for name in ("dX", "dW_gu", "dW_d", "dlogits"):
+        U.assert_rel(U.to_np(grads[name]), bwd[name], name)
+    # expert 0's rows alone (the segment that spans the most tiles)
+    lo, hi = fwd["offsets"][0], fwd["offsets"][1]
+    U.assert_rel(U.to_np(st.O)[lo:hi], fwd["O"][lo:hi], "O[expert 0]")
+    U.assert_rel(U.to_np(grads["dW_gu"])[0], bwd["dW_gu"][0], "dW_gu[expert 0]")
 
 
 def test_empty_experts_and_one_hot_expert():

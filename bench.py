@@ -68,6 +68,10 @@ def kernel_work(name, wl, lora_r=0):
         "route": T * E * 4 * 2 + T * k * 8,
         "router_bwd": T * E * 4 * 2 + T * k * 12 + P * 8 * ((I + 255) // 256),
         "permute_count": P * 4, "permute_scan": E * 8, "permute_scatter": P * 12,
+        # routing with the per-chunk expert counts (one byte per expert, rounded up to 16, per 32 tokens),
+        # then the scan-and-scatter kernel that reads those counts and the ids once and writes the permutation
+        "route_hist": T * E * 4 * 2 + T * k * 8 + -(-T // 32) * (-(-E // 16) * 16),
+        "permute_scan_scatter": -(-T // 32) * (-(-E // 16) * 16) + P * 4 + P * 8 + E * 8,
         # router Linear: X (bf16) and W_r (fp32) read once, logits / dW_r / dX written once
         "router_split_w": E * H * 4 + 3 * E * H * 2, "router_split_dlogits": T * E * 4 + 3 * T * E * 2,
         "gemm_router_logits": T * H * 2 + E * H * 4 + T * E * 4,
@@ -366,6 +370,51 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+def front_end_timing(B, logits, wl, bufs, dev, reps=200):
+    """Microseconds per call of the routing front end in CUDA-graph replay."""
+    perm = {n: bufs["perm"][n] for n in ("counts", "offsets", "sorted_pair", "pair_pos")}
+    idx, w, probs = bufs["topk_idx"], bufs["topk_w"], bufs["probs"]
+
+    def fused():
+        B.moe_route_permute(logits, wl.k, None, idx, w, probs, out=perm, ws=bufs["route_perm_ws"])
+
+    def two_calls():
+        B.moe_route(logits, wl.k, idx, w, probs)
+        B.moe_permute(idx, wl.E, None, out=perm, ws=bufs["perm_ws"])
+
+    graphs = {}
+    side = torch.cuda.Stream()
+    for name, fn in (("route_permute_us", fused), ("route_then_permute_us", two_calls)):
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs[name] = g
+    # three rounds, the two paths alternating; the median round of each
+    times = {name: [] for name in graphs}
+    for _ in range(3):
+        for name, g in graphs.items():
+            for _ in range(20):
+                g.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            times[name].append(a.elapsed_time(b) * 1e3 / reps)
+    out = {name: sorted(v)[1] for name, v in times.items()}
+    del graphs
+    out["note"] = (f"ids to permutation without the row gather, {reps} back-to-back CUDA-graph replays, median of "
+                   "3 alternating rounds; fused: "
+                   "moe_route_permute (2 kernels), two calls: moe_route + moe_permute (4 kernels)")
+    return out
+
+
 def workload_config(wl, args):
     return {"workload": f"{wl.name} MoE layer {'fwd+bwd' if wl.backward else 'fwd'}: T={wl.T} H={wl.H} "
                         f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else "")
@@ -408,6 +457,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-front-end", action="store_true", help="skip the routing front-end graph timing")
     ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling cases)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (scaled profiling cases: fewer experts, the same rows per expert with --tokens)")
@@ -628,6 +678,14 @@ def main():
             n_sus = int(max_over_ranks([n_sus], dev)[0])
         sus_ms, _ = timed_steps(profile=False, replay=graph is not None, nsteps=n_sus)
 
+    # Routing front end alone (ids -> permutation, no row gather), replayed
+    # from CUDA graphs back to back: the fused call (routing with the expert
+    # counts, then one scan-and-scatter kernel) and the two-call path
+    # (moe_route, then moe_permute's count, scan and scatter kernels).
+    front = None
+    if not args.no_front_end and rank == 0 and not rl:
+        front = front_end_timing(B, logits, wl, bufs, dev)
+
     # End to end through the public API with host buffers: every step copies
     # its inputs (X, logits, dY) from pinned host memory and reads its results
     # (Y, dX, dlogits) back. Inputs and outputs are double-buffered and the
@@ -805,7 +863,7 @@ def main():
             "note": "pinned host buffers; uploads/downloads on two copy streams overlap compute (the forward "
                     "starts once X and the logits are in, Y goes back during the backward); no L2 flush "
                     "(per-step working set >> L2)"},
-        "gpu_launches": launches, "clocks": clocks, "kernels": kernels,
+        "gpu_launches": launches, "clocks": clocks, "kernels": kernels, "front_end": front,
         "kernels_note": "value, ms_per_step and the roofline kernel come from the first timed pass (events "
                         "around the dominant kernel only); the per-kernel table from a second pass that records "
                         "every launch (serialised, and later under the power limit)",

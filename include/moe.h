@@ -114,6 +114,30 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
                 int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X, int H, moe_bf16* Xp, void* ws,
                 size_t ws_bytes, moe_stream_t stream);
 
+/* Bytes of workspace moe_route_permute needs for this problem size. */
+size_t moe_route_permute_workspace_bytes(int T, int E, int k);
+
+/*
+ * moe_route_permute -- moe_route followed by moe_permute in two kernels
+ * instead of five (plus the gather): the routing kernel also counts, per
+ * chunk of 32 tokens, how many of the chunk's pairs chose each expert, and
+ * one kernel turns those counts into counts/offsets and scatters the pairs.
+ * Source: fused-MoE Triton project summary (sourcepulse), Highlighted
+ * Details: softmax-topk fused with the expert indexing; the results are
+ * defined by moe_route and moe_permute above and are bit-identical to
+ * calling them in turn (topk_idx, topk_w, probs, counts, offsets,
+ * sorted_pair, pair_pos, Xp).
+ *
+ * Arguments as in moe_route and moe_permute (probs may be NULL; X and Xp
+ * both NULL skip the gather). ws >= moe_route_permute_workspace_bytes(T,E,k)
+ * bytes of device scratch (one byte per expert, rounded up to 16, per chunk
+ * of 32 tokens); MOE_ERR_WORKSPACE if smaller. Errors otherwise as the two
+ * calls; nothing is launched when an argument is rejected.
+ */
+int moe_route_permute(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w, float* probs,
+                      int32_t* counts, int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos,
+                      const moe_bf16* X, int H, moe_bf16* Xp, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /*
  * moe_permute_noalloc -- moe_permute without a workspace argument, for
  * callers that cannot allocate device memory: a host program or plug-in that

@@ -28,6 +28,9 @@ _SIGNATURES = {
     "moe_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_permute": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void, _c_void,
                              _c_int, _c_void, _c_void, _c_size, _c_void]),
+    "moe_route_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "moe_route_permute": (_c_int, [_c_void, _c_int, _c_int, _c_int] + [_c_void] * 7 + [_c_void, _c_int, _c_void,
+                                                                                     _c_void, _c_size, _c_void]),
     "moe_permute_noalloc": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void,
                                      _c_void, _c_int, _c_void, _c_void]),
     "moe_experts_fwd": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -161,6 +164,40 @@ def moe_permute(topk_idx: torch.Tensor, E: int, X: torch.Tensor | None = None, o
         _ptr(topk_idx), T, E, k, _ptr(o["counts"]), _ptr(o["offsets"]), _ptr(o["sorted_pair"]),
         _ptr(o["pair_pos"]), _ptr(X), H, _ptr(o.get("Xp")), _ptr(ws), ws.numel(), _stream(stream)))
     return o
+
+
+def moe_route_permute(logits: torch.Tensor, k: int, X: torch.Tensor | None = None, topk_idx=None, topk_w=None,
+                      probs=None, want_probs=True, out=None, ws=None, stream=None):
+    """moe_route then moe_permute in one call (two kernels plus the gather);
+    returns (topk_idx, topk_w, probs, perm) with perm as moe_permute's."""
+    T, E = logits.shape
+    dev = logits.device
+    _need(logits, torch.float32, (T, E), "logits")
+    P = T * k
+    topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty(T, k, dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    if probs is None and want_probs:
+        probs = torch.empty(T, E, dtype=torch.float32, device=dev)
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    o = dict(out or {})
+    o.setdefault("counts", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    o.setdefault("sorted_pair", torch.empty(P, dtype=torch.int32, device=dev))
+    o.setdefault("pair_pos", torch.empty(P, dtype=torch.int32, device=dev))
+    H = 0
+    if X is not None:
+        H = X.shape[1]
+        _need(X, torch.bfloat16, (T, H), "X")
+        o.setdefault("Xp", torch.empty(P, H, dtype=torch.bfloat16, device=dev))
+    need = lib().moe_route_permute_workspace_bytes(T, E, k)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("moe_route_permute", lib().moe_route_permute(
+        _ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _ptr(probs), _ptr(o["counts"]), _ptr(o["offsets"]),
+        _ptr(o["sorted_pair"]), _ptr(o["pair_pos"]), _ptr(X), H, _ptr(o.get("Xp")), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return topk_idx, topk_w, probs, o
 
 
 def moe_experts_fwd(Xp, offsets, sorted_pair, topk_w, T, E, k, W_gu, W_d, h=None, gu_save=None, O=None,

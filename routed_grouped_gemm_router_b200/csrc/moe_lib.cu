@@ -149,6 +149,8 @@ enum ProfSlot : int {
   kProfLoraDBGateUp,
   kProfLoraDADown,
   kProfLoraDBDown,
+  kProfRouteHist,
+  kProfPermScanScatter,
   kProfSlots
 };
 const char* const kProfNames[kProfSlots] = {
@@ -159,7 +161,7 @@ const char* const kProfNames[kProfSlots] = {
     "router_split_w", "gemm_router_logits",  "router_split_dlogits",   "gemm_router_wgrad",
     "router_sum_splits", "gemm_router_dgrad", "gemm_lora_z_gate_up", "gemm_lora_z_down", "gemm_lora_v_down",
     "gemm_lora_v_gate_up", "lora_weight_rows", "gemm_lora_da_gate_up", "gemm_lora_db_gate_up", "gemm_lora_da_down",
-    "gemm_lora_db_down"};
+    "gemm_lora_db_down", "route_hist", "permute_scan_scatter"};
 
 struct Profiler {
   std::mutex mu;
@@ -594,6 +596,64 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
   }
   if (gather) {
     ProfScope ps(kProfGatherX, stream);
+    const int64_t want = (P + 7) / 8;
+    const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
+    if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(X),
+                   static_cast<const int32_t*>(pair_pos), P, k, H / 8, reinterpret_cast<uint4*>(Xp)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+size_t moe_route_permute_workspace_bytes(int T, int E, int k) {
+  if (!shape_ok(T, E, k)) return 0;
+  return round256(static_cast<size_t>(route_hist_chunks(T)) * route_hist_ld(E));
+}
+
+int moe_route_permute(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w, float* probs,
+                      int32_t* counts, int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos, const moe_bf16* X,
+                      int H, moe_bf16* Xp, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  if (!ok_ptr(counts) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
+  const bool gather = (X != nullptr || Xp != nullptr);
+  if (gather && (!dims_ok(H) || (T > 0 && (!ok_ptr(X) || !ok_ptr(Xp))))) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!ok_ptr(logits) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_opt(probs) ||
+                !ok_ptr(sorted_pair) || !ok_ptr(pair_pos)))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_route_permute_workspace_bytes(T, E, k);
+  if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MOE_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  uint8_t* hist8 = static_cast<uint8_t*>(ws);
+  {
+    ProfScope ps(kProfRouteHist, stream);
+    if (launch_route_hist(logits, T, E, k, topk_idx, topk_w, probs, hist8, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  {
+    ProfScope ps(kProfPermScanScatter, stream);
+    const int nchunks = route_hist_chunks(T);
+    const size_t smem = scan_scatter_smem(E);
+    // always opted in: the kernel's static shared memory comes on top of this
+    if (cudaFuncSetAttribute(permute_scan_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_pdl(permute_scan_scatter_kernel, dim3(cdiv(nchunks, kScanScatterWarps)), dim3(kScanScatterThreads),
+                   smem, stream, static_cast<const uint8_t*>(hist8), route_hist_ld(E), nchunks,
+                   static_cast<const int32_t*>(topk_idx), T, E, k, counts, offsets, sorted_pair,
+                   pair_pos) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (gather) {
+    ProfScope ps(kProfGatherX, stream);
+    const int64_t P = static_cast<int64_t>(T) * k;
     const int64_t want = (P + 7) / 8;
     const int blocks = static_cast<int>(want < dev->num_sms * 16 ? want : dev->num_sms * 16);
     if (launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<const uint4*>(X),
@@ -1113,11 +1173,9 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   // 7. router logits gradient
   {
     ProfScope ps(kProfRouterBwd, stream);
-    int blocks = (T + 7) / 8;
-    if (blocks > dev->num_sms * 8) blocks = dev->num_sms * 8;
-    if (launch_pdl(router_bwd_kernel, dim3(blocks), dim3(256), sizeof(float) * 8 * E, stream, probs, topk_idx, topk_w,
-                   static_cast<const float*>(dw_part), pair_pos, kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k,
-                   dlogits) != cudaSuccess)
+    if (launch_router_bwd(probs, topk_idx, topk_w, static_cast<const float*>(dw_part), pair_pos,
+                          kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k, dlogits, dev->num_sms,
+                          stream) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   return MOE_OK;

@@ -1,7 +1,7 @@
 """The whole expert layer as a sequence of the C-ABI calls.
 
-``forward`` runs moe_route -> moe_permute -> moe_experts_fwd -> moe_combine
-and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. With
+``forward`` runs moe_route_permute (moe_route and moe_permute in one call)
+-> moe_experts_fwd -> moe_combine and returns Y plus the saved state; ``backward`` runs moe_layer_bwd. With
 gather=True the permute makes no Xp copy and the GEMMs read X and dY rows by
 token index (moe_experts_fwd_x / moe_layer_bwd_x): no Xp / dYp buffers
 (2 x T*k*H bf16 less memory), but the row-gather loads make those GEMMs
@@ -48,8 +48,10 @@ def forward(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d: torc
     preallocated outputs/workspaces (keys as in the returned state)."""
     b = bufs or {}
     T, E = logits.shape
-    idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
-    return _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather)
+    idx, w, probs, perm = B.moe_route_permute(logits, k, None if gather else X, b.get("topk_idx"), b.get("topk_w"),
+                                              b.get("probs"), out=b.get("perm"), ws=b.get("route_perm_ws"),
+                                              stream=stream)
+    return _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather, perm=perm)
 
 
 def forward_from_x(X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor, W_d: torch.Tensor, k: int,
@@ -66,8 +68,9 @@ def forward_from_x(X: torch.Tensor, W_r: torch.Tensor, W_gu: torch.Tensor, W_d: 
     return st
 
 
-def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather) -> LayerState:
-    perm = B.moe_permute(idx, E, None if gather else X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
+def _experts_forward(T, E, k, idx, w, probs, X, W_gu, W_d, save_gu, b, stream, gather, perm=None) -> LayerState:
+    if perm is None:
+        perm = B.moe_permute(idx, E, None if gather else X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
     h, gu, O = B.moe_experts_fwd(X if gather else perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k,
                                  W_gu, W_d, h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"), save_gu=save_gu,
                                  stream=stream, gather=gather)
@@ -81,8 +84,8 @@ def forward_lora(logits: torch.Tensor, X: torch.Tensor, W_gu: torch.Tensor, W_d:
     B_gu [E,2I,r], A_d [E,r,I], B_d [E,H,r] bf16, scale})."""
     b = bufs or {}
     T, E = logits.shape
-    idx, w, probs = B.moe_route(logits, k, b.get("topk_idx"), b.get("topk_w"), b.get("probs"), stream=stream)
-    perm = B.moe_permute(idx, E, X, out=b.get("perm"), ws=b.get("perm_ws"), stream=stream)
+    idx, w, probs, perm = B.moe_route_permute(logits, k, X, b.get("topk_idx"), b.get("topk_w"), b.get("probs"),
+                                              out=b.get("perm"), ws=b.get("route_perm_ws"), stream=stream)
     h, gu, O, Z_gu, Z_d = B.moe_experts_fwd_lora(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, T, E, k, W_gu,
                                                  W_d, lora, h=b.get("h"), gu_save=b.get("gu"), O=b.get("O"),
                                                  Z_gu=b.get("Z_gu"), Z_d=b.get("Z_d"), save_gu=save_gu,
@@ -152,6 +155,8 @@ def allocate(T: int, E: int, k: int, H: int, I: int, device, save_gu: bool = Tru
                   sorted_pair=torch.empty(P, dtype=torch.int32, device=device),
                   pair_pos=torch.empty(P, dtype=torch.int32, device=device)),
         perm_ws=torch.empty(max(lib.moe_permute_workspace_bytes(T, E, k), 1), dtype=torch.uint8, device=device),
+        route_perm_ws=torch.empty(max(lib.moe_route_permute_workspace_bytes(T, E, k), 1), dtype=torch.uint8,
+                                  device=device),
         h=torch.empty(P, I, dtype=bf, device=device),
         gu=torch.empty(P, 2 * I, dtype=bf, device=device) if save_gu else None,
         O=torch.empty(P, H, dtype=bf, device=device),

@@ -21,7 +21,8 @@ def test_profile_times_clock_and_results():
     clocks = {n: B.profile_read_clock(n) for n in prof}
     B.profile_enable(False)
     assert torch.equal(st0.Y, st1.Y) and all(torch.equal(g0[n], g1[n]) for n in g0)
-    for n in ("route", "permute_scatter", "gemm_fwd_gate_up", "gemm_bwd_wgrad_down", "combine_dx", "router_bwd"):
+    for n in ("route_hist", "permute_scan_scatter", "gemm_fwd_gate_up", "gemm_bwd_wgrad_down", "combine_dx",
+              "router_bwd"):
         assert n in prof and prof[n][0] > 0 and prof[n][1] >= 1, n
     for n, mhz in clocks.items():
         if n.startswith("gemm_"):

@@ -42,8 +42,10 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Algorithmic work per launch of each kernel, as a function of the workload:
-# GEMMs in flops (bf16 tensor cores), memory kernels in bytes (HBM).
-def kernel_work(name, wl, lora_r=0):
+# GEMMs in flops (bf16 tensor cores), memory kernels in bytes (HBM). A kernel
+# with both significant flops and bytes (dgrad through down) is reported
+# against whichever roofline bounds it on this workload (`peaks` given).
+def kernel_work(name, wl, lora_r=0, peaks=None):
     T, H, E, k, I, P = wl.T, wl.H, wl.E, wl.k, wl.I, wl.P
     r = lora_r
     flops = {
@@ -84,6 +86,11 @@ def kernel_work(name, wl, lora_r=0):
         "gemm_bwd_dgrad_down": (P * H * 2 + E * H * I * 2 + P * 2 * I * 2 + P * 2 * I * 2 + P * I * 2
                                 + P * 2 * ((I + 255) // 256) * 4 + (P * r * 2 + E * r * I * 2 if r else 0)),
     }
+    if name == "gemm_bwd_dgrad_down" and peaks is not None:
+        # dYp W_d per pair: 2 H I flops (plus the adapter's 2 H r)
+        fl = 2.0 * H * I * P + 2.0 * H * r * P
+        if fl / (peaks["bf16_tflops"] * 1e12) > nbytes[name] / (peaks["hbm_gbs"] * 1e9):
+            return "tensor", fl
     return "hbm", float(nbytes.get(name, 0))
 
 
@@ -415,6 +422,36 @@ def front_end_timing(B, logits, wl, bufs, dev, reps=200):
     return out
 
 
+def profile_ranges(B, layer, wl, X, logits, dY, W_gu, W_d, bufs):
+    """One layer step whose expert-GEMM call (moe_experts_fwd: gate/up then
+    down, each a one-CTA tail launch and a pair launch running side by side)
+    and whose backward call (moe_layer_bwd) each sit inside a profiler
+    start/stop range, for ncu's range replay: the DRAM bytes of a range are
+    those of its launches as they ran, concurrently."""
+    import torch.cuda.profiler as cuprof
+    b = bufs
+    idx, w, probs, perm = B.moe_route_permute(logits, wl.k, X, b["topk_idx"], b["topk_w"], b["probs"],
+                                              out=b["perm"], ws=b["route_perm_ws"])
+    torch.cuda.synchronize()
+    cuprof.start()
+    h, gu, O = B.moe_experts_fwd(perm["Xp"], perm["offsets"], perm["sorted_pair"], w, wl.T, wl.E, wl.k, W_gu, W_d,
+                                 h=b["h"], gu_save=b["gu"], O=b["O"], save_gu=True)
+    torch.cuda.synchronize()
+    cuprof.stop()
+    Y = B.moe_combine(O, perm["pair_pos"], wl.T, wl.k, Y=b["Y"])
+    st = layer.LayerState(wl.T, wl.E, wl.k, idx, w, probs, perm, h, gu, O, Y)
+    torch.cuda.synchronize()
+    cuprof.start()
+    layer.backward(st, dY, W_gu, W_d, bufs=b)
+    torch.cuda.synchronize()
+    cuprof.stop()
+    status = B.last_device_status()
+    print(json.dumps({"profile_ranges": ["moe_experts_fwd", "moe_layer_bwd"], "workload": wl.name,
+                      "device_status": status}), flush=True)
+    if status != 0:
+        raise RuntimeError(f"device status {B.status_str(status)}")
+
+
 def workload_config(wl, args):
     return {"workload": f"{wl.name} MoE layer {'fwd+bwd' if wl.backward else 'fwd'}: T={wl.T} H={wl.H} "
                         f"E={wl.E} k={wl.k} I={wl.I}" + (f" zipf_s={wl.zipf_s}" if wl.zipf_s else "")
@@ -458,6 +495,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-front-end", action="store_true", help="skip the routing front-end graph timing")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="after warm-up, run one step with the expert-GEMM call and the backward call inside "
+                         "profiler start/stop ranges (for ncu range replay), then exit")
     ap.add_argument("--tokens", type=int, default=None, help="override T (smaller profiling cases)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (scaled profiling cases: fewer experts, the same rows per expert with --tokens)")
@@ -582,6 +622,12 @@ def main():
     status = B.last_device_status()
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
+
+    if args.profile_range:
+        if rl or lr or gf or world > 1:
+            ap.error("--profile-range profiles the default layer on one GPU")
+        profile_ranges(B, layer, wl, X, logits, dY, W_gu, W_d, bufs)
+        return
 
     graph = None
     if args.cuda_graph:
@@ -797,7 +843,7 @@ def main():
     launches = 0
     for name, rec in prof.items():
         ms, n = rec[0], rec[1]
-        kind, work = kernel_work(name, wl, lr)
+        kind, work = kernel_work(name, wl, lr, peaks)
         avg_ms = ms / n
         launches += n
         rate = work / (avg_ms * 1e-3)
@@ -807,7 +853,7 @@ def main():
                          "unit": "TFLOP/s" if kind == "tensor" else "GB/s"}
         if len(rec) > 2:
             kernels[name]["sm_mhz_in_kernel"] = round(rec[2])
-    kind, work = kernel_work(dom, wl, lr)
+    kind, work = kernel_work(dom, wl, lr, peaks)
     avg_s = dom_prof[dom][0] / dom_prof[dom][1] * 1e-3
     if kind == "tensor":
         achieved = work / avg_s / 1e12

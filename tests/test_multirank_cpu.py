@@ -36,7 +36,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_rank_max_and_aggregate():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == [11.0, 20.0]

@@ -377,8 +377,10 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
-def front_end_timing(B, logits, wl, bufs, dev, reps=200):
-    """Microseconds per call of the routing front end in CUDA-graph replay."""
+def front_end_timing(B, logits, wl, bufs, dev, calls=20, reps=10):
+    """Microseconds per call of the routing front end: `calls` calls captured
+    in one CUDA graph (so the graph's own launch cost is shared), the graph
+    replayed `reps` times; median of three alternating rounds."""
     perm = {n: bufs["perm"][n] for n in ("counts", "offsets", "sorted_pair", "pair_pos")}
     idx, w, probs = bufs["topk_idx"], bufs["topk_w"], bufs["probs"]
 
@@ -399,26 +401,25 @@ def front_end_timing(B, logits, wl, bufs, dev, reps=200):
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn()
+            for _ in range(calls):
+                fn()
         graphs[name] = g
-    # three rounds, the two paths alternating; the median round of each
     times = {name: [] for name in graphs}
     for _ in range(3):
         for name, g in graphs.items():
-            for _ in range(20):
-                g.replay()
+            g.replay()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             for _ in range(reps):
                 g.replay()
             b.record()
             torch.cuda.synchronize()
-            times[name].append(a.elapsed_time(b) * 1e3 / reps)
+            times[name].append(a.elapsed_time(b) * 1e3 / (reps * calls))
     out = {name: sorted(v)[1] for name, v in times.items()}
     del graphs
-    out["note"] = (f"ids to permutation without the row gather, {reps} back-to-back CUDA-graph replays, median of "
-                   "3 alternating rounds; fused: "
-                   "moe_route_permute (2 kernels), two calls: moe_route + moe_permute (4 kernels)")
+    out["note"] = (f"ids to permutation without the row gather; {calls} calls per CUDA graph, {reps} replays, "
+                   "median of 3 alternating rounds; fused: moe_route_permute (2 kernels), two calls: moe_route + "
+                   "moe_permute (4 kernels)")
     return out
 
 

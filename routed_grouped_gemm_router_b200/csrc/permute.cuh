@@ -225,6 +225,16 @@ __global__ void __launch_bounds__(kScanScatterThreads) permute_scan_scatter_kern
   const int c0 = blockIdx.x * kScanScatterWarps;
   const int words = ld / 4;                               // ld is a multiple of 16, at most 1024
   const int groups = kScanScatterThreads / words;         // >= 1
+  // the ids this warp places in step 4 (k <= 32: lane j < k holds slot j of
+  // each of its chunk's 32 tokens), requested first: they depend on nothing
+  // computed here, so their latency overlaps the count-table sum
+  const int c = c0 + warp;
+  const int tc0 = c * 32;
+  const int tc1 = (tc0 + 32 < T) ? tc0 + 32 : T;
+  int ids[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    ids[i] = (k <= 32 && lane < k && tc0 + i < tc1) ? __ldg(flat + static_cast<int64_t>(tc0 + i) * k + lane) : 0;
 
   // 1. per expert: total over all chunks and the prefix before this block.
   // Thread (word wi, group g) reads 4 experts' bytes of chunks g, g + groups,
@@ -327,12 +337,9 @@ __global__ void __launch_bounds__(kScanScatterThreads) permute_scan_scatter_kern
   // order. The ids come from the routing kernel, so a token's k experts are
   // distinct: the lanes holding them bump distinct running counters, and
   // only consecutive tokens are ordered (by __syncwarp).
-  const int c = c0 + warp;
   if (c >= nchunks) return;
   int* run_w = s_run + warp * E;
   const int64_t P = static_cast<int64_t>(T) * k;
-  const int tc0 = c * 32;
-  const int tc1 = (tc0 + 32 < T) ? tc0 + 32 : T;
   auto place = [&](int64_t q, int e) {
     if (e < 0 || e >= E) {
       report(MOE_ERR_DEVICE_CHECK);
@@ -348,11 +355,6 @@ __global__ void __launch_bounds__(kScanScatterThreads) permute_scan_scatter_kern
     }
   };
   if (k <= 32) {
-    // lane j < k holds slot j of each of the chunk's 32 tokens, all requested at once
-    int ids[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      ids[i] = (lane < k && tc0 + i < tc1) ? __ldg(flat + static_cast<int64_t>(tc0 + i) * k + lane) : 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       if (tc0 + i >= tc1) break;

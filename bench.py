@@ -108,10 +108,10 @@ def read_peaks():
 _KERNEL_FILES = [
     (("gemm_router_", "router_split_", "router_sum_"), ["router_linear.cuh"]),
     (("gemm_",), ["grouped_gemm.cuh"]),
+    (("router_bwd",), ["router_bwd.cuh"]),  # before "route", which it starts with
     (("route",), ["route.cuh"]),
     (("permute_", "gather_"), ["permute.cuh"]),
     (("combine_",), ["combine.cuh"]),
-    (("router_bwd",), ["router_bwd.cuh"]),
 ]
 
 

@@ -229,6 +229,56 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Expert parallelism: the experts are split over ranks in contiguous blocks of
+ * experts_per_rank; each (token, expert) pair's row travels to the expert's
+ * owner, is computed there with moe_permute / moe_experts_fwd /
+ * moe_layer_bwd_pair_dw and comes back. The transport between ranks is the
+ * caller's (all-to-all); these calls prepare and finish the rows around it.
+ * Source: modelopt `moe` helpers, a2a_moe Flow: the pairs are expanded and
+ * sent to the experts, and the results come back to be weighted by the
+ * routing weights and summed per token.
+ *
+ * moe_ep_pack_rows -- for every expert-sorted row r (the rows of expert e are
+ * [offsets[e], offsets[e+1]) of a permutation made by moe_permute):
+ *   local_expert[r] = e % experts_per_rank  (its expert's index on the owner)
+ *   row_w[r]        = topk_w[sorted_pair[r]] (its routing weight)
+ * offsets [E+1], sorted_pair [T*k] int32 in; topk_w [T*k] fp32 in;
+ * local_expert [T*k] int32 out; row_w [T*k] fp32 out. E must be a multiple of
+ * experts_per_rank (else MOE_ERR_INVALID_ARG). Nothing is launched for T*k = 0.
+ */
+int moe_ep_pack_rows(const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w, int T, int E, int k,
+                     int experts_per_rank, int32_t* local_expert, float* row_w, moe_stream_t stream);
+
+/*
+ * moe_layer_bwd_pair_dw -- moe_layer_bwd without the router backward: in
+ * place of d logits it returns every pair's routing-weight gradient
+ *   dw[q] = <dY[q / k], o_q>,  o_q = the pair's unweighted expert output,
+ * summed in a fixed order. On an expert's owner rank it runs with k = 1 over
+ * the received rows (each row its own "token"; dY = the received dY rows), so
+ * dX and dw come back in the order the rows arrived.
+ * Arguments as moe_layer_bwd (probs, topk_idx and dlogits are not taken);
+ * dw [T*k] fp32 out; ws >= moe_layer_bwd_workspace_bytes(...).
+ */
+int moe_layer_bwd_pair_dw(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                          const float* topk_w, const int32_t* offsets, const int32_t* sorted_pair,
+                          const int32_t* pair_pos, int T, int E, int k, int H, int I, const moe_bf16* W_gu,
+                          const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d, float* dw, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_router_bwd_from_dw -- the router backward of moe_layer_bwd from
+ * routing-weight gradients given per expert-sorted row (dw_rows[r], r the
+ * row of pair q = pair_pos[q]), e.g. those returned by the experts' owners.
+ * Same formulas as moe_layer_bwd's d logits ("[WIP] Qwen3 MoE support",
+ * torchtune PR #2820, review comment: renormalisation by the top-k sum +
+ * 1e-20; then the softmax Jacobian). dw_rows [T*k], pair_pos [T*k], probs
+ * [T,E], topk_idx / topk_w [T,k] in; dlogits [T,E] fp32 out.
+ */
+int moe_router_bwd_from_dw(const float* dw_rows, const int32_t* pair_pos, const float* probs,
+                           const int32_t* topk_idx, const float* topk_w, int T, int E, int k, float* dlogits,
+                           moe_stream_t stream);
+
+/*
  * moe_layer_bwd with fp32 weight gradients: dW_gu [E,2I,H] and dW_d [E,H,I]
  * are fp32, the wgrad GEMMs' fp32 accumulators stored without rounding
  * (moe_layer_bwd rounds the same accumulators to bf16, so rounding this

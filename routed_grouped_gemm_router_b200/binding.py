@@ -31,6 +31,10 @@ _SIGNATURES = {
     "moe_route_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
     "moe_route_permute": (_c_int, [_c_void, _c_int, _c_int, _c_int] + [_c_void] * 7 + [_c_void, _c_int, _c_void,
                                                                                      _c_void, _c_size, _c_void]),
+    "moe_ep_pack_rows": (_c_int, [_c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_void, _c_void,
+                                  _c_void]),
+    "moe_layer_bwd_pair_dw": (_c_int, [_c_void] * 8 + [_c_int] * 5 + [_c_void] * 6 + [_c_void, _c_size, _c_void]),
+    "moe_router_bwd_from_dw": (_c_int, [_c_void] * 5 + [_c_int] * 3 + [_c_void, _c_void]),
     "moe_permute_noalloc": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void,
                                      _c_void, _c_int, _c_void, _c_void]),
     "moe_experts_fwd": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -336,6 +340,53 @@ def moe_layer_bwd(dY, Xp, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_p
     else:
         _check(name, getattr(lib(), name)(*head, *tail))
     return o
+
+
+def moe_ep_pack_rows(offsets, sorted_pair, topk_w, T, E, k, experts_per_rank, out=None, stream=None):
+    """Per expert-sorted row: its expert's index on the owner rank and its
+    routing weight; returns (local_expert [T*k] int32, row_w [T*k] fp32)."""
+    P = T * k
+    dev = offsets.device
+    o = dict(out or {})
+    le = o.get("local_expert", torch.empty(P, dtype=torch.int32, device=dev))
+    rw = o.get("row_w", torch.empty(P, dtype=torch.float32, device=dev))
+    _check("moe_ep_pack_rows", lib().moe_ep_pack_rows(_ptr(offsets), _ptr(sorted_pair), _ptr(topk_w), T, E, k,
+                                                      experts_per_rank, _ptr(le), _ptr(rw), _stream(stream)))
+    return le, rw
+
+
+def moe_layer_bwd_pair_dw(dY, Xp, gu_save, h, topk_w, offsets, sorted_pair, pair_pos, T, E, k, W_gu, W_d,
+                          out=None, ws=None, stream=None):
+    """moe_layer_bwd returning each pair's routing-weight gradient (out["dw"]
+    [T*k] fp32) in place of d logits; returns the dict of dX, dW_gu, dW_d, dw."""
+    H = W_gu.shape[2]
+    I = W_d.shape[2]
+    dev = dY.device
+    o = dict(out or {})
+    o.setdefault("dX", torch.empty(T, H, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW_gu", torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW_d", torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dw", torch.empty(T * k, dtype=torch.float32, device=dev))
+    need = lib().moe_layer_bwd_workspace_bytes(T, E, k, H, I, 1 if gu_save is None else 0)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("moe_layer_bwd_pair_dw", lib().moe_layer_bwd_pair_dw(
+        _ptr(dY), _ptr(Xp), _ptr(gu_save), _ptr(h), _ptr(topk_w), _ptr(offsets), _ptr(sorted_pair), _ptr(pair_pos),
+        T, E, k, H, I, _ptr(W_gu), _ptr(W_d), _ptr(o["dX"]), _ptr(o["dW_gu"]), _ptr(o["dW_d"]), _ptr(o["dw"]),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_router_bwd_from_dw(dw_rows, pair_pos, probs, topk_idx, topk_w, dlogits=None, stream=None):
+    """d logits from routing-weight gradients given per expert-sorted row."""
+    T, E = probs.shape
+    k = topk_idx.shape[1]
+    if dlogits is None:
+        dlogits = torch.empty(T, E, dtype=torch.float32, device=probs.device)
+    _check("moe_router_bwd_from_dw", lib().moe_router_bwd_from_dw(
+        _ptr(dw_rows), _ptr(pair_pos), _ptr(probs), _ptr(topk_idx), _ptr(topk_w), T, E, k, _ptr(dlogits),
+        _stream(stream)))
+    return dlogits
 
 
 def _router_ws(T, H, E, dev, ws):

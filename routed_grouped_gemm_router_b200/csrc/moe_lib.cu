@@ -2,7 +2,8 @@
 //
 // This file validates arguments, sizes the caller's workspace, encodes the TMA
 // tensor maps and enqueues the kernels of route.cuh, permute.cuh,
-// grouped_gemm.cuh, combine.cuh and router_bwd.cuh on the caller's stream.
+// grouped_gemm.cuh, combine.cuh, router_bwd.cuh and ep.cuh on the caller's
+// stream.
 // It allocates no device memory and never synchronises (except the status
 // read and the profiling read, which say so).
 #include <cuda.h>
@@ -17,6 +18,7 @@
 #include "../../include/moe.h"
 #include "combine.cuh"
 #include "common.cuh"
+#include "ep.cuh"
 #include "grouped_gemm.cuh"
 #include "lora.cuh"
 #include "permute.cuh"
@@ -151,6 +153,8 @@ enum ProfSlot : int {
   kProfLoraDBDown,
   kProfRouteHist,
   kProfPermScanScatter,
+  kProfPairDw,
+  kProfEpPack,
   kProfSlots
 };
 const char* const kProfNames[kProfSlots] = {
@@ -161,7 +165,7 @@ const char* const kProfNames[kProfSlots] = {
     "router_split_w", "gemm_router_logits",  "router_split_dlogits",   "gemm_router_wgrad",
     "router_sum_splits", "gemm_router_dgrad", "gemm_lora_z_gate_up", "gemm_lora_z_down", "gemm_lora_v_down",
     "gemm_lora_v_gate_up", "lora_weight_rows", "gemm_lora_da_gate_up", "gemm_lora_db_gate_up", "gemm_lora_da_down",
-    "gemm_lora_db_down", "route_hist", "permute_scan_scatter"};
+    "gemm_lora_db_down", "route_hist", "permute_scan_scatter", "pair_dw", "ep_pack_rows"};
 
 struct Profiler {
   std::mutex mu;
@@ -892,7 +896,7 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
                    const int32_t* offsets, const int32_t* sorted_pair, const int32_t* pair_pos, int T, int E, int k,
                    int H, int I, const moe_bf16* W_gu, const moe_bf16* W_d, moe_bf16* dX, void* dW_gu, void* dW_d,
                    bool dw_f32, bool accumulate, float* dlogits, void* ws, size_t ws_bytes, cudaStream_t stream,
-                   const LoraArgs* lora = nullptr) {
+                   const LoraArgs* lora = nullptr, bool pair_dw_out = false, float* pair_dw = nullptr) {
   const moe_bf16* Xp = src;
   if (!shape_ok(T, E, k) || !dims_ok(H) || !dims_ok(I)) return MOE_ERR_INVALID_ARG;
   if (lora != nullptr) {
@@ -905,9 +909,14 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
   }
   if (!ok_ptr(offsets)) return MOE_ERR_INVALID_ARG;
   const int64_t P = static_cast<int64_t>(T) * k;
-  if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_opt(h) || !ok_ptr(probs) ||
-                !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(sorted_pair) || !ok_ptr(pair_pos) ||
-                !ok_ptr(W_gu) || !ok_ptr(W_d) || !ok_ptr(dX) || !ok_ptr(dlogits)))
+  // pair_dw_out: the routing-weight gradient of every pair (pair_dw [T*k])
+  // is the output in place of the router backward (probs, topk_idx and
+  // dlogits unused)
+  const bool router = !pair_dw_out;
+  if (P > 0 && (!ok_ptr(dY) || !ok_ptr(Xp) || !ok_opt(gu_save) || !ok_opt(h) || !ok_ptr(topk_w) ||
+                !ok_ptr(sorted_pair) || !ok_ptr(pair_pos) || !ok_ptr(W_gu) || !ok_ptr(W_d) || !ok_ptr(dX)))
+    return MOE_ERR_INVALID_ARG;
+  if (P > 0 && (router ? (!ok_ptr(probs) || !ok_ptr(topk_idx) || !ok_ptr(dlogits)) : !ok_ptr(pair_dw)))
     return MOE_ERR_INVALID_ARG;
   if (P > 0 && lora != nullptr && (!ok_ptr(lora->Z_gu) || !ok_ptr(lora->Z_d))) return MOE_ERR_INVALID_ARG;
   (void)h;  // not read: the dgrad-down epilogue recomputes h = silu(g) * u from g|u
@@ -1170,12 +1179,19 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
       if (int st = launch_gemm<kBwdWgrad>(g, pair_grid(tiles, dev->num_sms), stream, w.slot)) return st;
     }
   }
-  // 7. router logits gradient
-  {
+  // 7. router logits gradient, or each pair's routing-weight gradient
+  if (router) {
     ProfScope ps(kProfRouterBwd, stream);
     if (launch_router_bwd(probs, topk_idx, topk_w, static_cast<const float*>(dw_part), pair_pos,
                           kDwSlotsPerNTile * nt_dgrad_down, static_cast<int64_t>(T), E, k, dlogits, dev->num_sms,
                           stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  } else {
+    ProfScope ps(kProfPairDw, stream);
+    const int64_t want = (P + 255) / 256;
+    const int blocks = static_cast<int>(want < dev->num_sms * 8 ? want : dev->num_sms * 8);
+    if (launch_pdl(pair_dw_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<const float*>(dw_part), pair_pos,
+                   kDwSlotsPerNTile * nt_dgrad_down, P, pair_dw) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   return MOE_OK;
@@ -1192,6 +1208,49 @@ int moe_layer_bwd(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_sav
                   float* dlogits, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return layer_bwd_impl(dY, Xp, false, gu_save, h, probs, topk_idx, topk_w, offsets, sorted_pair, pair_pos, T, E, k,
                         H, I, W_gu, W_d, dX, dW_gu, dW_d, false, false, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_layer_bwd_pair_dw(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,
+                          const float* topk_w, const int32_t* offsets, const int32_t* sorted_pair,
+                          const int32_t* pair_pos, int T, int E, int k, int H, int I, const moe_bf16* W_gu,
+                          const moe_bf16* W_d, moe_bf16* dX, moe_bf16* dW_gu, moe_bf16* dW_d, float* dw, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  return layer_bwd_impl(dY, Xp, false, gu_save, h, nullptr, nullptr, topk_w, offsets, sorted_pair, pair_pos, T, E,
+                        k, H, I, W_gu, W_d, dX, dW_gu, dW_d, false, false, nullptr, ws, ws_bytes, stream, nullptr,
+                        true, dw);
+}
+
+int moe_router_bwd_from_dw(const float* dw_rows, const int32_t* pair_pos, const float* probs,
+                           const int32_t* topk_idx, const float* topk_w, int T, int E, int k, float* dlogits,
+                           moe_stream_t stream) {
+  if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!ok_ptr(dw_rows) || !ok_ptr(pair_pos) || !ok_ptr(probs) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) ||
+      !ok_ptr(dlogits))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  ProfScope ps(kProfRouterBwd, stream);
+  if (launch_router_bwd(probs, topk_idx, topk_w, dw_rows, pair_pos, 1, static_cast<int64_t>(T), E, k, dlogits,
+                        dev->num_sms, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_ep_pack_rows(const int32_t* offsets, const int32_t* sorted_pair, const float* topk_w, int T, int E, int k,
+                     int experts_per_rank, int32_t* local_expert, float* row_w, moe_stream_t stream) {
+  if (!shape_ok(T, E, k) || experts_per_rank < 1 || E % experts_per_rank != 0) return MOE_ERR_INVALID_ARG;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (P == 0) return MOE_OK;
+  if (!ok_ptr(offsets) || !ok_ptr(sorted_pair) || !ok_ptr(topk_w) || !ok_ptr(local_expert) || !ok_ptr(row_w))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev;
+  if (int st = current_device_info(&dev)) return st;
+  ProfScope ps(kProfEpPack, stream);
+  if (launch_pdl(ep_pack_rows_kernel, dim3(E), dim3(256), 0, stream, offsets, sorted_pair, topk_w, P,
+                 experts_per_rank, local_expert, row_w) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 int moe_layer_bwd_dw_f32(const moe_bf16* dY, const moe_bf16* Xp, const moe_bf16* gu_save, const moe_bf16* h,

@@ -466,7 +466,9 @@ def workload_config(wl, args):
             "lora_rank": int(getattr(args, "lora", 0)),
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I, "seed": args.seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)",
-            "parallelism": (f"dp{args.gpus} (own batch per rank, weight gradients summed over NCCL: "
+            "parallelism": (f"ep{args.gpus} (own batch per rank, E/{args.gpus} experts per rank, rows to their "
+                            "owners and back by all-to-all over NCCL)" if getattr(args, "ep", False) else
+                            f"dp{args.gpus} (own batch per rank, weight gradients summed over NCCL: "
                             f"{getattr(args, 'grad_sync', 'allreduce')})" if args.gpus > 1 and wl.backward
                             and getattr(args, "grad_sync", "allreduce") != "none"
                             else f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU")}
@@ -491,6 +493,9 @@ def main():
                     help="include the router Linear (logits = X W_r^T and its backward) in the step")
     ap.add_argument("--grad-sync", default="allreduce", choices=["allreduce", "reduce_scatter", "none"],
                     help="N > 1: how the ranks' weight gradients are summed after each backward (NCCL)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallel: each rank owns E/N experts, rows travel to their owners and back "
+                         "(all-to-all over NCCL); with one GPU a one-rank group")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -530,12 +535,31 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    ep_mode = args.ep
+    if ep_mode and (args.router_linear or args.lora or args.gather_fused or args.dw_f32 or args.cuda_graph
+                    or not wl.backward):
+        ap.error("--ep runs the default layer forward + backward, eagerly")
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    elif ep_mode:  # one rank: the exchange is the rank's copy to itself
+        import socket
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(port))
+        dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
 
     # every rank its own batch: seed + rank
     inp = make_inputs(wl, seed=args.seed + rank, with_dy=wl.backward)
-    X, W_gu, W_d = inp.X.to(dev), inp.W_gu.to(dev), inp.W_d.to(dev)
+    if ep_mode:
+        # expert parallel: this rank holds only its block of experts
+        from routed_grouped_gemm_router_b200 import ep as EP
+        e_lo, e_hi = EP.experts_of_rank(wl.E, world, rank)
+        X, W_gu, W_d = inp.X.to(dev), inp.W_gu[e_lo:e_hi].to(dev), inp.W_d[e_lo:e_hi].to(dev)
+    else:
+        X, W_gu, W_d = inp.X.to(dev), inp.W_gu.to(dev), inp.W_d.to(dev)
     logits = inp.logits.to(dev)
     W_r = inp.W_r.to(dev)
     dY = inp.dY.to(dev) if wl.backward else None
@@ -558,7 +582,7 @@ def main():
     # are summed over the ranks after every backward (one NCCL collective),
     # timed on its own with events around it.
     grad_flat, grad_extra, sync_evs = None, [], []
-    sync = world > 1 and wl.backward and args.grad_sync != "none"
+    sync = world > 1 and wl.backward and args.grad_sync != "none" and not ep_mode
     if sync and args.cuda_graph:
         ap.error("--cuda-graph captures one rank's step; the N > 1 step with its gradient exchange runs eagerly")
     if sync:
@@ -585,6 +609,8 @@ def main():
 
     def run_fwd(X_, logits_, b):
         """The layer's forward through the public API."""
+        if ep_mode:
+            return EP.ep_forward(logits_, X_, W_gu, W_d, wl.k, wl.E)
         if rl:
             return layer.forward_from_x(X_, W_r, W_gu, W_d, wl.k, bufs=b, gather=gf)
         if lr:
@@ -593,6 +619,8 @@ def main():
 
     def run_bwd(st, dY_, X_, b):
         """The layer's backward through the public API."""
+        if ep_mode:
+            return EP.ep_backward(st, dY_, W_gu, W_d)
         if rl:
             return layer.backward_to_x(st, dY_, X_, W_r, W_gu, W_d, bufs=b)
         if lr:
@@ -625,7 +653,7 @@ def main():
         raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
 
     if args.profile_range:
-        if rl or lr or gf or world > 1:
+        if rl or lr or gf or world > 1 or ep_mode:
             ap.error("--profile-range profiles the default layer on one GPU")
         profile_ranges(B, layer, wl, X, logits, dY, W_gu, W_d, bufs)
         return
@@ -829,7 +857,7 @@ def main():
         total_ms, e2e_ms = t_max, (e_max if e2e_ms is not None else None)
         sus_total = s_max if sus_ms else None
     if rank != 0:
-        if world > 1:
+        if dist.is_initialized():
             dist.destroy_process_group()
         return
 
@@ -931,7 +959,7 @@ def main():
                     "between steps outside the events"},
     }
     print(json.dumps(line), flush=True)
-    if world > 1:
+    if dist.is_initialized():
         dist.destroy_process_group()
 
 

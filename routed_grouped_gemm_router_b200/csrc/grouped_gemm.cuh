@@ -166,13 +166,19 @@ struct GemmParams {
   // out_ld = M), so that a product with few rows can be computed as its
   // transpose with the few rows as narrow columns.
   int out_transposed;
+  // bf16 wgrad: write full 32 x 32 chunks with TMA stores through tmOut
+  // ([E * M rows, N] bf16, 32 x 32 boxes, 64-byte swizzle: the staging
+  // buffer's layout) instead of per-thread stores.
+  int out_tma;
+  CUtensorMap tmOut;
 };
 
 template <int CG>
 __host__ __device__ inline size_t gemm_smem_bytes(int E) {
   return 1024 /*alignment slack*/ + static_cast<size_t>(CgCfg<CG>::kStages) * CgCfg<CG>::kStageBytes +
          kNumBarriers * 8 + 16 +
-         2 * static_cast<size_t>(E + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * kStageWarpBytes;
+         2 * static_cast<size_t>(E + 1) * 4 + 512 /*staging alignment*/ +
+         static_cast<size_t>(kEpiWarps) * kStageWarpBytes;
 }
 
 struct TileInfo {
@@ -390,7 +396,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
   int* s_tstart = s_off + (p.E + 1);
-  uint8_t* s_stage = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 15) & ~uintptr_t(15));
+  // staging buffers 512-byte aligned: the 64-byte swizzle of the TMA stores
+  // takes its pattern from the shared-memory address bits
+  uint8_t* s_stage = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (p.E + 1)) + 511) &
+                                                ~uintptr_t(511));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -990,6 +999,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             continue;
           }
           float v[32];
+          if (kWgrad && p.out_tma) {
+            // bf16 weight gradient through TMA stores: the chunk is staged
+            // once in the store box's layout and one thread stores it; a
+            // partial box (fewer than 32 rows left in dW[e]) goes the
+            // per-thread way, which must not overlap a store still reading
+            // the buffer either
+            const bool full = wrows == 32;
+            const int row_g = ti.e * p.M + static_cast<int>(wrow0);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if (!(hh == 0 ? in0 : in1)) continue;  // warp-uniform
+              const uint32_t* a = hh == 0 ? a0 : a1;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a[j]);
+              if (lane == 0) bulk_wait_group_read0();
+              __syncwarp();
+              if (full) {
+                stage_row(stg, lane, v);
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(&p.tmOut, stg, col0 + 32 * hh, row_g);
+                  bulk_commit_group();
+                }
+              } else {
+                emit_chunk(stg, v, out_base, wrow0, p.out_ld, col0 + 32 * hh, p.N, wrows, tr_row, tr_q, lane);
+              }
+            }
+            continue;
+          }
           if (in0) {  // warp-uniform
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = wq * __uint_as_float(a0[j]);
@@ -1017,6 +1056,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       }
       ++tcount;
     }
+    // this warp's TMA stores are complete before the CTA leaves
+    if (kWgrad && p.out_tma && lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------- tear-down

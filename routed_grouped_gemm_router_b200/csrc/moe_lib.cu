@@ -26,6 +26,12 @@
 #include "router_bwd.cuh"
 #include "router_linear.cuh"
 
+// bf16 weight gradients leave the wgrad epilogue through TMA stores (0: per-
+// thread stores from the staging buffer, as the other outputs).
+#ifndef MOE_WGRAD_TMA_STORE
+#define MOE_WGRAD_TMA_STORE 1
+#endif
+
 namespace moe {
 
 // Waits on an mbarrier that nothing ever arrives at, with the library's
@@ -106,7 +112,8 @@ EncodeTiledFn encode_fn() {
 // box_inner x box_rows; out-of-range elements read as zero.
 // row_stride_elems (0: = inner) is the distance between rows in elements.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
-              uint32_t box_rows, uint64_t row_stride_elems = 0) {
+              uint32_t box_rows, uint64_t row_stride_elems = 0,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -114,7 +121,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1090,6 +1097,11 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wg.m_tiles = cdiv(2 * I, kBM);
     wg.n_tiles = cdiv(H, kBN);
     set_dw_out(wg, dW_gu, dw_f32, accumulate);
+    if (!dw_f32 && MOE_WGRAD_TMA_STORE) {  // bf16 dW: full 32 x 32 chunks leave through TMA stores
+      if (!make_map(&wg.tmOut, dW_gu, H, static_cast<uint64_t>(E) * 2 * I, 32, 32, 0, CU_TENSOR_MAP_SWIZZLE_64B))
+        return MOE_ERR_CUDA;
+      wg.out_tma = 1;
+    }
     wg.out_ld = H;
     wg.out_expert_stride = static_cast<int64_t>(2) * I * H;
     const int64_t tiles = static_cast<int64_t>(E) * wg.m_tiles * wg.n_tiles;
@@ -1117,6 +1129,11 @@ int layer_bwd_impl(const moe_bf16* dY, const moe_bf16* src, bool gather, const m
     wd.m_tiles = cdiv(H, kBM);
     wd.n_tiles = cdiv(I, kBN);
     set_dw_out(wd, dW_d, dw_f32, accumulate);
+    if (!dw_f32 && MOE_WGRAD_TMA_STORE) {
+      if (!make_map(&wd.tmOut, dW_d, I, static_cast<uint64_t>(E) * H, 32, 32, 0, CU_TENSOR_MAP_SWIZZLE_64B))
+        return MOE_ERR_CUDA;
+      wd.out_tma = 1;
+    }
     wd.out_ld = I;
     wd.out_expert_stride = static_cast<int64_t>(H) * I;
     const int64_t tiles = static_cast<int64_t>(E) * wd.m_tiles * wd.n_tiles;

@@ -305,22 +305,33 @@ inline int rowgrouped_grid(int64_t P, int E, int n_tiles, int num_sms) {
   return pair_grid((static_cast<int64_t>(cdiv(P, kBM)) + E) * n_tiles, num_sms);
 }
 // CTAs (even) for the one-CTA tail instance, from the expected work split:
-// about 0.65 E segments end in a tail of 1..128 rows (half of them for
-// evenly spread routing, more when a few experts take most rows and the
-// rest are small), one CTA for one tile time each; the full tiles cost two
-// CTAs each (P / 256 of them). When the average segment is 128 rows or less
-// nearly every tile is a tail.
-#ifndef MOE_TAIL_WEIGHT
-#define MOE_TAIL_WEIGHT 0.65
+// about w E segments end in a tail of 1..128 rows (half of them for evenly
+// spread routing, more when a few experts take most rows and the rest are
+// small), one CTA for one tile time each; the full tiles cost two CTAs each
+// (P / 256 of them). When the average segment is 128 rows or less nearly
+// every tile is a tail. The weight w also carries the tail tiles' lower
+// efficiency per CTA (each stages all 256 B rows), and its best value grows
+// with the segment length: measured 0.65 on 512-row segments (Qwen3-30B-A3B
+// layer, 0.4-1.0 swept) and 0.8 on 1024-row ones (Qwen3-235B-A22B layer,
+// 0.5-1.0 swept); in between it is interpolated. MOE_TAIL_WEIGHT fixes it.
+inline double tail_weight(int64_t P, int E) {
+#ifdef MOE_TAIL_WEIGHT
+  (void)P;
+  (void)E;
+  return MOE_TAIL_WEIGHT;
+#else
+  const double rows = static_cast<double>(P) / E;
+  const double f = rows <= 512.0 ? 0.0 : rows >= 1024.0 ? 1.0 : (rows - 512.0) / 512.0;
+  return 0.65 + 0.15 * f;
 #endif
-constexpr double kTailWeight = MOE_TAIL_WEIGHT;
+}
 inline int tail_ctas(int64_t P, int E, int num_sms) {
   if (!kTailTiles || P == 0) return 0;
   int c;
   if (P <= static_cast<int64_t>(128) * E) {
     c = num_sms - 4;
   } else {
-    const double tail = kTailWeight * E, full = 2.0 * static_cast<double>(P) / kBM;
+    const double tail = tail_weight(P, E) * E, full = 2.0 * static_cast<double>(P) / kBM;
     c = static_cast<int>(num_sms * tail / (tail + full) + 0.5);
   }
   c &= ~1;

@@ -61,6 +61,11 @@ typedef enum {
   MOE_ERR_DEVICE_CHECK = 6
 } moe_status;
 
+/* Number of kernels this library has launched (enqueued) in this process so
+ * far, on every stream and device; a launch recorded into a CUDA graph counts
+ * once, when it is captured. */
+unsigned long long moe_launch_count(void);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_str(int status);
 

@@ -23,6 +23,7 @@ _c_size = ctypes.c_size_t
 
 _SIGNATURES = {
     "moe_status_str": (ctypes.c_char_p, [_c_int]),
+    "moe_launch_count": (ctypes.c_ulonglong, []),
     "moe_last_device_status": (_c_int, [_c_void]),
     "moe_route": (_c_int, [_c_void, _c_int, _c_int, _c_int, _c_void, _c_void, _c_void, _c_void]),
     "moe_permute_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int]),
@@ -126,6 +127,11 @@ def _need(t: torch.Tensor, dtype, shape, name):
     if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
         raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().moe_launch_count())
 
 
 def last_device_status(stream=None) -> int:

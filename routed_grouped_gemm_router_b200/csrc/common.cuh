@@ -1,5 +1,6 @@
 // Shared device helpers: the device status word, bf16 packing, warp utilities.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <utility>
 #include <cuda_bf16.h>
@@ -48,6 +49,13 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
   return v;
 }
 
+// Kernels this library has launched in the process (every launch goes
+// through launch_pdl_clustered; read with moe_launch_count).
+inline std::atomic<unsigned long long>& launch_count() {
+  static std::atomic<unsigned long long> n{0};
+  return n;
+}
+
 // Launches `kernel` on stream `s` with programmatic stream serialisation, so
 // its set-up may overlap the tail of the previous kernel on the stream (the
 // kernel itself waits for that kernel's results, see griddep_wait).
@@ -72,7 +80,9 @@ inline cudaError_t launch_pdl_clustered(void (*kernel)(KArgs...), dim3 grid, dim
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cluster_x > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (err == cudaSuccess) launch_count().fetch_add(1, std::memory_order_relaxed);
+  return err;
 }
 
 template <typename... KArgs, typename... Args>

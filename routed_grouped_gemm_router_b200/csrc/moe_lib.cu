@@ -548,6 +548,8 @@ const char* moe_status_str(int status) {
   }
 }
 
+unsigned long long moe_launch_count(void) { return launch_count().load(std::memory_order_relaxed); }
+
 int moe_last_device_status(moe_stream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0;
@@ -1464,6 +1466,7 @@ int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream) {
   DeviceInfo* dev;
   if (int st = current_device_info(&dev)) return st;
   wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  launch_count().fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
 

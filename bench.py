@@ -45,7 +45,37 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # GEMMs in flops (bf16 tensor cores), memory kernels in bytes (HBM). A kernel
 # with both significant flops and bytes (dgrad through down) is reported
 # against whichever roofline bounds it on this workload (`peaks` given).
-def kernel_work(name, wl, lora_r=0, peaks=None):
+def gemm_bytes(name, wl, lora_r=0, active=None):
+    """Algorithmic bytes of one expert GEMM call of the layer (with g|u saved
+    in the forward): each operand row read once, the weights of the experts
+    that have rows (``active``; all E when not given) read once, each output
+    written once. The weight gradients write all E experts (zeros for idle
+    ones). None for kernels that are not expert GEMMs."""
+    T, H, E, k, I, P = wl.T, wl.H, wl.E, wl.k, wl.I, wl.P
+    r = lora_r
+    Ea = E if active is None else active
+    w_gu, w_d = Ea * 2 * I * H * 2, Ea * H * I * 2
+    # with adapters the row-grouped GEMMs also read Z (P r) and B (r N per expert)
+    z = (lambda n: P * r * 2 + Ea * r * n * 2) if r else (lambda n: 0)
+    part = P * 2 * ((I + 255) // 256) * 4          # routing-weight partials of the dgrad through down
+    table = {
+        "gemm_fwd_gate_up": P * H * 2 + w_gu + P * I * 2 + P * 2 * I * 2 + z(2 * I),
+        "gemm_recompute_gate_up": P * H * 2 + w_gu + P * 2 * I * 2 + z(2 * I),
+        "gemm_fwd_down": P * I * 2 + w_d + P * 4 + P * H * 2 + z(H),
+        # dYp, W_d and g|u read; dGU, w*h and the partials written
+        "gemm_bwd_dgrad_down": P * H * 2 + w_d + P * 2 * I * 2 + P * 2 * I * 2 + P * I * 2 + part + z(I),
+        "gemm_bwd_dgrad_gate_up": P * 2 * I * 2 + w_gu + P * H * 2 + z(H),
+        "gemm_bwd_wgrad_gate_up": P * H * 2 + P * 2 * I * 2 + E * 2 * I * H * 2,
+        "gemm_bwd_wgrad_down": P * H * 2 + P * I * 2 + E * H * I * 2,
+    }
+    return table.get(name)
+
+
+def kernel_work(name, wl, lora_r=0, peaks=None, active=None):
+    """(bound, work) of one launch of kernel ``name``: FLOPs for a tensor-bound
+    kernel, bytes for an HBM-bound one. With ``peaks`` an expert GEMM takes the
+    bound whose time at the measured peak is the longer (a decode-sized batch
+    streams the active experts' weights and is HBM-bound)."""
     T, H, E, k, I, P = wl.T, wl.H, wl.E, wl.k, wl.I, wl.P
     r = lora_r
     flops = {
@@ -62,6 +92,10 @@ def kernel_work(name, wl, lora_r=0, peaks=None):
         "gemm_lora_da_down": 2.0 * I * r * P, "gemm_lora_db_down": 2.0 * H * r * P,
     }
     if name in flops:
+        gb = gemm_bytes(name, wl, r, active)
+        if peaks is not None and gb is not None and \
+                gb / (peaks["hbm_gbs"] * 1e9) > flops[name] / (peaks["bf16_tflops"] * 1e12):
+            return "hbm", float(gb)
         return "tensor", flops[name]
     nbytes = {
         # one read of each source row (L2 serves the k re-reads), one write per pair row
@@ -80,11 +114,9 @@ def kernel_work(name, wl, lora_r=0, peaks=None):
         "gemm_router_wgrad": T * H * 2 + T * E * 4 + E * H * 4, "router_sum_splits": 2 * E * H * 4,
         "gemm_router_dgrad": T * E * 4 + E * H * 4 + 2 * T * H * 2,
         "lora_weight_rows": 2 * P * r * 2 + P * 8,
-        # dgrad through down is HBM-bound by its roofline (these bytes at the
-        # measured copy bandwidth take longer than its flops at the bf16 peak):
-        # dYp, W_d and g|u read; dGU, w*h and the routing-weight partials written
-        "gemm_bwd_dgrad_down": (P * H * 2 + E * H * I * 2 + P * 2 * I * 2 + P * 2 * I * 2 + P * I * 2
-                                + P * 2 * ((I + 255) // 256) * 4 + (P * r * 2 + E * r * I * 2 if r else 0)),
+        # dgrad through down: HBM-bound on the narrower layers (its bytes at the
+        # measured copy bandwidth take longer than its flops at the bf16 peak)
+        "gemm_bwd_dgrad_down": gemm_bytes("gemm_bwd_dgrad_down", wl, r, active),
     }
     if name == "gemm_bwd_dgrad_down" and peaks is not None:
         # dYp W_d per pair: 2 H I flops (plus the adapter's 2 H r)
@@ -651,6 +683,10 @@ def main():
     status = B.last_device_status()
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
+    # experts that received rows: whose weights the row-grouped GEMMs read
+    active = None
+    if not ep_mode and bufs.get("perm") is not None:
+        active = int((bufs["perm"]["counts"] > 0).sum().item())
 
     if args.profile_range:
         if rl or lr or gf or world > 1 or ep_mode:
@@ -876,7 +912,7 @@ def main():
     kernels = {}
     for name, rec in prof.items():
         ms, n = rec[0], rec[1]
-        kind, work = kernel_work(name, wl, lr, peaks)
+        kind, work = kernel_work(name, wl, lr, peaks, active)
         avg_ms = ms / n
         rate = work / (avg_ms * 1e-3)
         kernels[name] = {"ms_per_step": ms / args.steps, "launches": n, "share": ms / sum(prof_step_ms),
@@ -885,7 +921,7 @@ def main():
                          "unit": "TFLOP/s" if kind == "tensor" else "GB/s"}
         if len(rec) > 2:
             kernels[name]["sm_mhz_in_kernel"] = round(rec[2])
-    kind, work = kernel_work(dom, wl, lr, peaks)
+    kind, work = kernel_work(dom, wl, lr, peaks, active)
     avg_s = dom_prof[dom][0] / dom_prof[dom][1] * 1e-3
     if kind == "tensor":
         achieved = work / avg_s / 1e12
@@ -913,7 +949,7 @@ def main():
     same_kernels = not (lr or args.dw_f32 or gf)
     traffic, traffic_src = measured_traffic(dom, wl.name) if same_kernels else (None, None)
     roof.update({"kernel": dom, "traffic": traffic, "traffic_source": traffic_src,
-                 "algorithmic_per_launch": work,
+                 "algorithmic_per_launch": work, "experts_with_rows": active,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 
     cpu = None

@@ -21,6 +21,27 @@ def test_dgrad_down_bound_follows_the_workload():
     assert bench.kernel_work("gemm_fwd_gate_up", wl)[1] == 4.0 * wl.H * wl.I * wl.P
 
 
+def test_decode_sized_batch_is_hbm_bound():
+    """64 tokens: the expert GEMMs stream the active experts' weights, so each
+    takes the HBM bound with those bytes; the big layers keep the tensor bound."""
+    wl = WORKLOADS["zipf-t64"]
+    names = ("gemm_fwd_gate_up", "gemm_fwd_down", "gemm_bwd_dgrad_gate_up", "gemm_bwd_dgrad_down",
+             "gemm_bwd_wgrad_gate_up", "gemm_bwd_wgrad_down")
+    for name in names:
+        kind, work = bench.kernel_work(name, wl, 0, PEAKS, active=90)
+        assert kind == "hbm", name
+        assert work == bench.gemm_bytes(name, wl, 0, 90)
+    H, I, P, E = wl.H, wl.I, wl.P, wl.E
+    # gate/up forward: X rows in, the 90 experts' [W_g; W_u] in, h and g|u out
+    assert bench.gemm_bytes("gemm_fwd_gate_up", wl, 0, 90) == P * H * 2 + 90 * 2 * I * H * 2 + P * I * 2 + P * 4 * I
+    # the weight gradient writes every expert's block, idle ones included
+    assert bench.gemm_bytes("gemm_bwd_wgrad_down", wl, 0, 90) == P * H * 2 + P * I * 2 + E * H * I * 2
+    for wname in ("qwen3-235b-a22b", "gpt-oss-20b"):
+        for name in names:
+            assert bench.kernel_work(name, WORKLOADS[wname], 0, PEAKS)[0] == "tensor", (wname, name)
+    assert bench.gemm_bytes("gather_x", wl) is None
+
+
 def test_traffic_from_committed_summaries():
     t235, src235 = bench.measured_traffic("gemm_bwd_wgrad_gate_up", "qwen3-235b-a22b")
     t16, src16 = bench.measured_traffic("gemm_bwd_wgrad_gate_up", "qwen3-235b-a22b-e16-t2048")

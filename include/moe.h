@@ -156,8 +156,8 @@ int moe_route_permute(const float* logits, int T, int E, int k, int32_t* topk_id
  * problem must satisfy ceil(T*k / 2048) * E <= 262144 (for E = 128: up to
  * 4,194,304 pairs); larger problems return MOE_ERR_WORKSPACE and launch
  * nothing. The first call on a device looks up that array's device address
- * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. The address is kept for the life of the process: after
+ * (cudaGetSymbolAddress) with the device current. The address is kept for the
+ * life of the process: after
  * cudaDeviceReset (or anything else that destroys and re-creates the device's
  * context) it is stale, so do not call this entry point again in that
  * process. All calls share the array: calls whose executions

@@ -96,6 +96,15 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 #ifndef MOE_STREAM_STORES
 #define MOE_STREAM_STORES 1
 #endif
+// dgrad through down: how many 32-column chunks ahead of its use the
+// epilogue loads g|u into registers. 1 (the default) fits the 168 registers a
+// thread of the 320-thread CTA gets; 2 spills 48 bytes and measured 2-7 %
+// slower on this kernel.
+#ifndef MOE_DGRAD_GU_AHEAD
+#define MOE_DGRAD_GU_AHEAD 1
+#endif
+constexpr int kGuAhead = MOE_DGRAD_GU_AHEAD;
+static_assert(kGuAhead == 1 || kGuAhead == 2, "g|u loads run 1 or 2 chunks ahead");
 // Raster of the row-grouped tiles inside an expert: 0 = N block fastest
 // (concurrent pairs share A rows), 1 = row block fastest (concurrent pairs
 // share a weight tile).
@@ -846,14 +855,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           wq = (q >= 0 && q < p.P) ? __ldg(p.topk_w + q) : 0.0f;
         }
       }
-      // dgrad-down: issue the first chunk's g/u/h loads before the wait so
-      // their latency hides behind the main loop
-      // g/u of the first two chunks are requested before the wait; each later
-      // chunk two chunks ahead of its use
+      // dgrad-down: g|u of the first kGuAhead chunks are requested before
+      // the wait, so their latency hides behind the main loop; each later
+      // chunk's kGuAhead chunks ahead of its use
       uint4 dd_cur[8], dd_nxt[8];
       if constexpr (KIND == kBwdDgradDown) {
         dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + ch0 * 32 + tr_q * 8, tr_row, dd_cur);
-        dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + (ch0 + 1) * 32 + tr_q * 8, tr_row, dd_nxt);
+        if constexpr (kGuAhead == 2)
+          dgrad_down_load(p, wrow0, wrows, ti.n_blk * kBN + (ch0 + 1) * 32 + tr_q * 8, tr_row, dd_nxt);
       }
 
       const int acc = tcount & 1;
@@ -900,7 +909,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
           const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
           uint4 nxt2[8];
-          if (ch + 2 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 64, tr_row, nxt2);
+          if constexpr (kGuAhead == 2) {
+            if (ch + 2 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 64, tr_row, nxt2);
+          } else {
+            if (ch + 1 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 32, tr_row, dd_nxt);
+          }
           uint32_t a[32];
           tmem_ld_32x32b_x32(taddr + ch * 32, a);
           tmem_ld_wait();
@@ -937,7 +950,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             dd_cur[x] = dd_nxt[x];
-            dd_nxt[x] = nxt2[x];
+            if constexpr (kGuAhead == 2) dd_nxt[x] = nxt2[x];
           }
         }
         // each row's partial dot product is spread over the 4 lanes with the

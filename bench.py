@@ -126,6 +126,20 @@ def kernel_work(name, wl, lora_r=0, peaks=None, active=None):
     return "hbm", float(nbytes.get(name, 0))
 
 
+# Datasheet figures per B200, reported beside the measured denominators: dense
+# bf16 tensor throughput (without 2:4 sparsity) and HBM3e bandwidth.
+DATASHEET_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+
+def datasheet_fracs(roof):
+    """The roofline's achieved rate against the datasheet peak of its bound
+    (None for a bound the datasheet does not cover)."""
+    key = {"tensor": "bf16_tflops", "hbm": "hbm_gbs"}.get(roof["bound"])
+    if key is None:
+        return None, None
+    return DATASHEET_PEAKS[key], roof["achieved"] / DATASHEET_PEAKS[key]
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -948,6 +962,7 @@ def main():
     # gradients and gathered operands change what the GEMMs move
     same_kernels = not (lr or args.dw_f32 or gf)
     traffic, traffic_src = measured_traffic(dom, wl.name) if same_kernels else (None, None)
+    roof["peak_datasheet"], roof["frac_datasheet"] = datasheet_fracs(roof)
     roof.update({"kernel": dom, "traffic": traffic, "traffic_source": traffic_src,
                  "algorithmic_per_launch": work, "experts_with_rows": active,
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
@@ -970,6 +985,7 @@ def main():
         "config": workload_config(wl, args),
         "tokens_per_s": world * wl.T * args.steps / (total_ms * 1e-3),
         "pct_of_bf16_peak": value / world / peaks["bf16_tflops"],
+        "pct_of_bf16_peak_datasheet": value / world / DATASHEET_PEAKS["bf16_tflops"],
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": None if e2e_ms is None else {
             "value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

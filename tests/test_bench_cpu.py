@@ -83,3 +83,11 @@ def test_config_labels():
     rep = bench.workload_config(wl, argparse.Namespace(gpus=4, grad_sync="none", **base))
     assert rep["parallelism"] == "replicas x4"
     assert bench.aggregate_tflops(2, 1e12, 10, 1000.0) == 20.0
+
+
+def test_datasheet_fractions():
+    """The datasheet denominators sit beside the measured ones: 2.25 PFLOP/s
+    dense bf16 for a tensor-bound kernel, 8 TB/s for an HBM-bound one."""
+    assert bench.datasheet_fracs({"bound": "tensor", "achieved": 1125.0}) == (2250.0, 0.5)
+    assert bench.datasheet_fracs({"bound": "hbm", "achieved": 6000.0}) == (8000.0, 0.75)
+    assert bench.datasheet_fracs({"bound": "alu", "achieved": 1.0}) == (None, None)

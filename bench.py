@@ -140,6 +140,18 @@ def datasheet_fracs(roof):
     return DATASHEET_PEAKS[key], roof["achieved"] / DATASHEET_PEAKS[key]
 
 
+def routing_stats(counts):
+    """The realised expert histogram of a batch (rows per expert): largest
+    segment, experts with no rows, mean rows per expert and the Gini
+    coefficient of the row counts (0 = every expert the same, (E-1)/E = one
+    expert takes every row)."""
+    c = sorted(int(x) for x in counts)
+    n, tot = len(c), sum(c)
+    gini = 0.0 if tot == 0 else 2.0 * sum((i + 1) * x for i, x in enumerate(c)) / (n * tot) - (n + 1) / n
+    return {"max_rows": c[-1] if c else 0, "empty_experts": sum(1 for x in c if x == 0),
+            "mean_rows": tot / n if n else 0.0, "gini": gini}
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -698,9 +710,10 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {B.status_str(status)}")
     # experts that received rows: whose weights the row-grouped GEMMs read
-    active = None
+    active, routing = None, None
     if not ep_mode and bufs.get("perm") is not None:
         active = int((bufs["perm"]["counts"] > 0).sum().item())
+        routing = routing_stats(bufs["perm"]["counts"].cpu().tolist())
 
     if args.profile_range:
         if rl or lr or gf or world > 1 or ep_mode:
@@ -993,6 +1006,7 @@ def main():
             "note": "pinned host buffers; uploads/downloads on two copy streams overlap compute (the forward "
                     "starts once X and the logits are in, Y goes back during the backward); no L2 flush "
                     "(per-step working set >> L2)"},
+        "routing": routing,
         "gpu_launches": head_launches, "clocks": clocks, "kernels": kernels, "front_end": front,
         "kernels_note": "value, ms_per_step and the roofline kernel come from the first timed pass (events "
                         "around the dominant kernel only); the per-kernel table from a second pass that records "

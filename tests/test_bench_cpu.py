@@ -91,3 +91,14 @@ def test_datasheet_fractions():
     assert bench.datasheet_fracs({"bound": "tensor", "achieved": 1125.0}) == (2250.0, 0.5)
     assert bench.datasheet_fracs({"bound": "hbm", "achieved": 6000.0}) == (8000.0, 0.75)
     assert bench.datasheet_fracs({"bound": "alu", "achieved": 1.0}) == (None, None)
+
+
+def test_routing_stats():
+    even = bench.routing_stats([4, 4, 4, 4])
+    assert even == {"max_rows": 4, "empty_experts": 0, "mean_rows": 4.0, "gini": 0.0}
+    one = bench.routing_stats([0, 0, 0, 12])
+    assert one["max_rows"] == 12 and one["empty_experts"] == 3 and abs(one["gini"] - 0.75) < 1e-12
+    # brute force: mean absolute difference over all pairs / (2 * mean)
+    c = [3, 0, 7, 1, 9]
+    mad = sum(abs(a - b) for a in c for b in c) / len(c) ** 2
+    assert abs(bench.routing_stats(c)["gini"] - mad / (2 * sum(c) / len(c))) < 1e-12

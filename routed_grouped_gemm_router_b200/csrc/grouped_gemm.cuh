@@ -908,7 +908,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 #pragma unroll 1
         for (int ch = ch0; ch < ch0 + kChunks; ++ch) {
           const int col = ti.n_blk * kBN + ch * 32 + tr_q * 8;
-          uint4 nxt2[8];
+          [[maybe_unused]] uint4 nxt2[8];  // used when kGuAhead == 2
           if constexpr (kGuAhead == 2) {
             if (ch + 2 < ch0 + kChunks) dgrad_down_load(p, wrow0, wrows, col + 64, tr_row, nxt2);
           } else {

@@ -206,7 +206,10 @@ namespace moe {
 // of the block's chunks before w, and the warp places its chunk's pairs in
 // ascending pair order, so each expert's rows keep ascending pair ids: the
 // stable argsort of the flat ids. The ids must come from routing (each token's k
-// experts distinct), as in moe_route_permute.
+// experts distinct), as in moe_route_permute. Block width, measured with the
+// routing kernel before it: 4 warps is much slower (each block sums the whole
+// table with fewer threads); 16 warps take a whole SM's registers, so its
+// blocks cannot start beside the routing kernel's and end no sooner.
 constexpr int kScanScatterWarps = 8;
 constexpr int kScanScatterThreads = 32 * kScanScatterWarps;
 

@@ -33,8 +33,11 @@
  *    MOE_ERR_INVALID_ARG, a workspace that is too small MOE_ERR_WORKSPACE, a
  *    device that is not sm_100 MOE_ERR_UNSUPPORTED, a failed launch
  *    MOE_ERR_CUDA. Problems found on the device (an expert id outside [0,E),
- *    a pipeline wait that exceeded its time limit) are recorded in a device
- *    status word that moe_last_device_status reads; kernels never trap.
+ *    segment bounds `offsets` given to a GEMM call that are not
+ *    0 <= offsets[0] <= ... <= offsets[E] <= T*k, a pipeline wait that
+ *    exceeded its time limit) are recorded in a device status word that
+ *    moe_last_device_status reads; kernels never trap. A GEMM given such
+ *    offsets computes no tile (a weight gradient is written as zeros).
  *  - Limits: 1 <= k <= E <= 1024, T >= 0 (T == 0 is a valid empty batch),
  *    T*k < 2^31, H and I positive multiples of 8 (16-byte rows).
  */
@@ -72,7 +75,8 @@ const char* moe_status_str(int status);
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MOE_OK, MOE_ERR_TIMEOUT (a kernel wait ran out and the
  * kernel unwound) or MOE_ERR_DEVICE_CHECK (an expert id outside [0,E) was
- * skipped). MOE_ERR_CUDA if the synchronisation itself failed. */
+ * skipped, or a GEMM refused its segment bounds). MOE_ERR_CUDA if the
+ * synchronisation itself failed. */
 int moe_last_device_status(moe_stream_t stream);
 
 /*

@@ -459,6 +459,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   griddep_launch_dependents();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = p.offsets[i];
   __syncthreads();
+  // The segment bounds come from the caller. Unless 0 <= offsets[0] <= ... <=
+  // offsets[E] <= P, tiles would reach rows outside the operands: such a call
+  // runs no tile (every segment emptied; a weight gradient writes zeros) and
+  // reports MOE_ERR_DEVICE_CHECK.
+  {
+    int bad = 0;
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+      const int v = s_off[i];
+      bad |= (v < 0) | (static_cast<int64_t>(v) > p.P) | (i < p.E && v > s_off[i + 1]);
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) report(MOE_ERR_DEVICE_CHECK);
+      for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_off[i] = 0;
+      __syncthreads();
+    }
+  }
   if (warp == 0 && !kWgrad) {
     // pair tiles of expert e = ceil(rows_e / 256) * n_tiles; exclusive prefix over experts
     const int per = (p.E + 31) / 32;

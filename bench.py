@@ -981,7 +981,7 @@ def main():
                  "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"})
 
     cpu = None
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline is timed at N = 1 only
         lo = lora_np(wl, args) if lr else None
         sample, ts, es, lo = cpu_sample(inp, wl, target_s=args.cpu_target_s, router=rl, lora=lo)
         t0 = time.perf_counter()
